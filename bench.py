@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Benchmark: split-KV varlen GQA decode on B200, achieved HBM GB/s and us/call.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload long|ragged|continuous|shortq|tiny]
+
+One step = one attention call over one batch of the workload (plan made once,
+the call captured once in a CUDA graph and replayed).  Inputs are resident in
+HBM; L2 is flushed (a 512 MB write) before every timed step, outside the
+timed events.  Bytes counted per call are the algorithmic ones: K and V over
+the actual ragged lengths plus Q and O (lse is reported apart).  With N > 1
+(torchrun) every rank runs its own copy of the workload (independent
+sequences: weak scaling, no collective on the data path) and the time is the
+max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0
+only), on a bounded sample of the same workload per step.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "achieved HBM GB/s and µs/call, varlen GQA split-KV decode, 1×B200 (% of roofline)"
+FLUSH_BYTES = 512 << 20
+
+DESCRIPTIONS = {
+    "long": "low-parallelism long-context decode: B=1, q_len=1, Hq=64, Hkv=8, D=128, kv=32768",
+    "ragged": "ragged decode batch: B=64, q_len=1, Hq=32, Hkv=8, D=128, kv~U{0..8192}",
+    "continuous": "continuous batching: B=256, q_len=1, Hq=64, Hkv=8, D=128, kv~lognormal(mean 2048, "
+                  "sigma 1) in [1,16384], step 0",
+    "shortq": "short-query varlen: B=32, q_len~U{1..16}, Hq=32, Hkv=4, D=128, kv~U{q_len..4096}, causal",
+    "tiny": "tiny decode: B=2, q_len=1, Hq=4, Hkv=1, D=64, kv={37,100}",
+}
+
+
+def algorithmic_bytes(batch: W.Batch) -> dict:
+    sh = batch.shape
+    kv = int(batch.lens_k.sum()) * sh.Hkv * sh.D * 2 * 2
+    tq = int(batch.lens_q.sum())
+    qo = tq * sh.Hq * sh.D * 2 * 2
+    return {"kv": kv, "qo": qo, "total": kv + qo, "lse": tq * sh.Hq * 4}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running
+    (reads only; changes no setting)."""
+
+    REASONS = {0x2: "applications_clocks", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.reasons = 0
+        self.sm_max = None
+        self.err = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                idx = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() else device_index
+                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nvml, self._h = pynvml, h
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that, do not guess
+            self._nvml = None
+            self.err = f"nvml unavailable: {e}"
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _reasons_now(self):
+        n = self._nvml
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(n, fn):
+                return getattr(n, fn)(self._h)
+        return 0
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons_now())
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nvml:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nvml:
+            self._t.join(timeout=2)
+
+    def summary(self) -> dict:
+        d = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+             "sm_max_mhz": self.sm_max, "samples": len(self.samples),
+             "reasons": [name for bit, name in self.REASONS.items() if self.reasons & bit],
+             "source": "nvml, sampled every 10 ms during the timed region"}
+        if self.err:
+            d["error"] = self.err
+        return d
+
+
+# ------------------------------------------------------------------ peaks / profiles
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
+    except Exception:
+        return 6650.0, "fallback 6.65 TB/s (pool measurement)"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "varlen_gqa_split_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, when it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None, "no ncu record"
+    e = rec.get(workload)
+    if not e:
+        return None, "no ncu record for this workload"
+    if e.get("source_hash") != kernel_source_hash():
+        return None, "kernel changed since the ncu capture"
+    if e.get("kernel") != kernel:
+        return None, "ncu record names another kernel"
+    return int(e["dram_bytes_per_launch"]), e.get("note", "")
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    return rank, world, local, pg
+
+
+def max_over_ranks(x: float, pg) -> float:
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ------------------------------------------------------------------ reference arm (oracle)
+
+def run_reference(args, batch: W.Batch) -> dict:
+    """The oracle as it stands, timed on the host cores: each step computes a
+    random sample of the workload's output rows, sized so that warm-up plus
+    timed steps take about VGQA_REF_BUDGET_S seconds (default 120)."""
+    import oracle
+    sh = batch.shape
+    qb, kb, vb = W.bits(batch.q), W.bits(batch.k), W.bits(batch.v)
+    lens_q, lens_k = batch.lens_q, batch.lens_k
+    rows_all = np.array([(b, qi, h) for b in range(len(lens_q)) for qi in range(int(lens_q[b]))
+                         for h in range(sh.Hq)], dtype=np.int64)
+    # algorithmic bytes of a row: its share of its sequence's K/V for its KV
+    # head (read by G * Lq rows) plus its q and out rows
+    row_bytes = np.array([lens_k[b] * sh.D * 4 / (sh.G * max(int(lens_q[b]), 1)) + sh.D * 4
+                          for b in rows_all[:, 0]])
+    budget_s = float(os.environ.get("VGQA_REF_BUDGET_S", "120"))
+    t0 = time.perf_counter()
+    oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, rows_all[:1], B=sh.B, Hq=sh.Hq,
+                          Hkv=sh.Hkv, D=sh.D, causal=sh.causal)
+    t_row = max(time.perf_counter() - t0, 1e-5)
+    n_steps = args.steps + args.warmup
+    per_step = max(1, min(len(rows_all), int(budget_s / n_steps / t_row)))
+    rng = np.random.default_rng(0)
+    times, nbytes = [], []
+    for s in range(n_steps):
+        pick = rng.choice(len(rows_all), size=per_step, replace=False)
+        t0 = time.perf_counter()
+        oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, rows_all[pick], B=sh.B, Hq=sh.Hq,
+                              Hkv=sh.Hkv, D=sh.D, causal=sh.causal)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            nbytes.append(float(row_bytes[pick].sum()))
+    total_t = sum(times)
+    value = sum(nbytes) / total_t / 1e9
+    sample = (f"{per_step} of {len(rows_all)} output rows (b, qi, h) per step, drawn at random; "
+              f"bytes attributed per row (K/V share + q + out)")
+    return {
+        "metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": DESCRIPTIONS[args.workload], "kind": "fp64 CPU oracle (oracle/oracle.c)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def cpu_baseline(batch: W.Batch, bytes_: dict, budget_s: float = 20.0) -> dict:
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    same workload, scaled to GB/s of the workload's algorithmic bytes."""
+    import oracle
+    sh = batch.shape
+    qb, kb, vb = W.bits(batch.q), W.bits(batch.k), W.bits(batch.v)
+    lens_q, lens_k = batch.lens_q, batch.lens_k
+    rows_all = np.array([(b, qi, h) for b in range(len(lens_q)) for qi in range(int(lens_q[b]))
+                         for h in range(sh.Hq)], dtype=np.int64)
+    # work per row ~ its visible keys; sample whole rows until the budget is met
+    t0 = time.perf_counter()
+    oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, rows_all[:8], B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv,
+                          D=sh.D, causal=sh.causal)
+    t8 = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(len(rows_all), max(8, 8 * (budget_s / 3) / t8)))
+    rng = np.random.default_rng(1)
+    sel = rows_all if n >= len(rows_all) else rows_all[np.sort(rng.choice(len(rows_all), n, replace=False))]
+    ts = []
+    for _ in range(3):
+        t0 = time.perf_counter()
+        oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, sel, B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv,
+                              D=sh.D, causal=sh.causal)
+        ts.append(time.perf_counter() - t0)
+    t = statistics.median(ts)
+    # scale: the sample's share of the workload's (row x key) work
+    vis = lambda b: int(lens_k[b])  # noqa: E731  (q_len rows see <= Lk keys; decode sees Lk)
+    work_sel = sum(vis(b) for b in sel[:, 0])
+    work_all = sum(vis(b) for b in rows_all[:, 0])
+    frac = work_sel / max(work_all, 1)
+    value = bytes_["total"] * frac / t / 1e9
+    return {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(sel)} of {len(rows_all)} output rows ({100 * frac:.1f}% of the row x key work), "
+                      f"median of 3, scaled to the whole call"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def make_inputs(name: str, device):
+    batch = W.workload(name, seed=0, gen_device=device)
+    return batch
+
+
+def run_ours(args, rank, world, local, pg) -> dict | None:
+    from varlen_gqa_split_b200 import Plan, build
+    build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    batch = make_inputs(args.workload, dev)
+    sh = batch.shape
+    bytes_ = algorithmic_bytes(batch)
+    q, k, v = batch.q, batch.k, batch.v
+    cu_q = torch.from_numpy(batch.cu_q).to(dev)
+    cu_k = torch.from_numpy(batch.cu_k).to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], sh.Hq, dtype=torch.float32, device=dev)
+    plan = Plan(sh.B, sh.s_max, sh.Hq, sh.Hkv, sh.D, sh.max_q, nsplit=args.nsplit, variant=args.variant,
+                stages=args.stages, combine=args.combine)
+    info = plan.info
+    launches_per_call = 2 if info["combine"] == 1 else 1
+
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        plan.run(q, k, v, cu_q, cu_k, out, lse)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="global"):
+            plan.run(q, k, v, cu_q, cu_k, out, lse)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev0=None, ev1=None):
+        flush.zero_()
+        if ev0 is not None:
+            ev0.record(stream)
+        graph.replay()
+        if ev1 is not None:
+            ev1.record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+        stream.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(pg)
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as clocks:
+            for e0, e1 in evs:
+                step(e0, e1)
+            stream.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier(pg)
+    per_step_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    total_ms = max_over_ranks(sum(per_step_ms), pg)
+    ms_per_step = total_ms / args.steps
+    value = bytes_["total"] * args.steps * world / (total_ms * 1e-3) / 1e9
+    assert plan.check_error() == 0, "device error flag set during the benchmark"
+
+    # roofline of the split kernel: with a fused merge (or one split) the call
+    # is that one launch, so its event time is the kernel's
+    peak, peak_src = measured_peak()
+    kernel = {1: "split_simt_kernel", 2: "split_mma_kernel"}[info["variant"]]
+    mean_kernel_ms = sum(per_step_ms) / len(per_step_ms)
+    if launches_per_call == 1:
+        achieved = bytes_["total"] / (mean_kernel_ms * 1e-3) / 1e9
+        traffic, traffic_note = recorded_traffic(args.workload, kernel)
+        roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                    "algorithmic_bytes_per_launch": bytes_["total"]}
+        if traffic is None:
+            roofline["traffic_note"] = traffic_note
+    else:
+        roofline = {"bound": "hbm", "kernel": kernel, "achieved": None, "peak": peak, "unit": "GB/s",
+                    "frac": None, "traffic": None,
+                    "note": "separate combine kernel: the split kernel is not timed alone"}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = max(3, min(args.steps, 20))
+        hq = batch.q.cpu().pin_memory()
+        hk = batch.k.cpu().pin_memory()
+        hv = batch.v.cpu().pin_memory()
+        hcq = torch.from_numpy(batch.cu_q).pin_memory()
+        hck = torch.from_numpy(batch.cu_k).pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        hl = torch.empty(hq.shape[0], sh.Hq, dtype=torch.float32).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dcq, dck = torch.empty_like(cu_q), torch.empty_like(cu_k)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        with torch.cuda.stream(stream):
+            def e2e_step():
+                dq.copy_(hq, non_blocking=True)
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                dcq.copy_(hcq, non_blocking=True)
+                dck.copy_(hck, non_blocking=True)
+                o, l_ = plan.run(dq, dk, dv, dcq, dck, out, lse)
+                ho.copy_(o, non_blocking=True)
+                hl.copy_(l_, non_blocking=True)
+            for _ in range(2):
+                e2e_step()
+            stream.synchronize()
+            barrier(pg)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            e1.record(stream)
+            stream.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg)
+        e2e = {"value": bytes_["total"] * n_e2e * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "us_per_call": 1e3 * e2e_ms / n_e2e}
+
+    res = None
+    if rank == 0:
+        cpu = None if (args.no_cpu_baseline or world > 1) else cpu_baseline(batch, bytes_)
+        res = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_call": 1e3 * ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": DESCRIPTIONS[args.workload], "B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv,
+                       "D": sh.D, "max_q": sh.max_q, "s_max": sh.s_max,
+                       "kv_tokens": int(batch.lens_k.sum()), "q_tokens": int(batch.lens_q.sum()),
+                       "bytes_per_call": bytes_["total"], "lse_bytes_per_call": bytes_["lse"],
+                       "l2": "flushed before every timed step (512 MB write, outside the timed events)",
+                       "timing": "CUDA events around each CUDA-graph replay of one attn_run, summed",
+                       "parallelism": f"replicas x{world} (independent sequences)",
+                       "plan": {kk: info[kk] for kk in ("variant", "nsplit", "chunk", "stages", "grid_x",
+                                                         "grid_y", "grid_z", "combine", "smem_bytes")}},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_call * args.steps,
+            "clocks": clocks.summary(),
+            "per_step_us": {"min": 1e3 * min(per_step_ms), "median": 1e3 * statistics.median(per_step_ms),
+                            "max": 1e3 * max(per_step_ms)},
+        }
+    del graph
+    plan.close()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(DESCRIPTIONS), default="long")
+    ap.add_argument("--nsplit", type=int, default=0)
+    ap.add_argument("--variant", type=int, default=0)
+    ap.add_argument("--stages", type=int, default=0)
+    ap.add_argument("--combine", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        batch = make_inputs(args.workload, "cpu")
+        res = run_reference(args, batch)
+        print(json.dumps(res), flush=True)
+        return
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    try:
+        res = run_ours(args, rank, world, local, pg)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

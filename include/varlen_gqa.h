@@ -1,0 +1,195 @@
+/*
+ * varlen_gqa.h -- C ABI of the B200 (sm_100a) split-KV varlen GQA attention
+ * library (libvgqa.so).
+ *
+ * The library computes grouped-query attention for packed variable-length
+ * (THD) batches in the decode and short-query regime:
+ *
+ *   for each sequence b, query token qi < Lq_b and query head h
+ *   (hk = h / G, G = Hq / Hkv, n = clamp(Lk_b - Lq_b + qi + 1, 0, Lk_b)):
+ *     s_j = (1/sqrt(D)) q[cu_q[b]+qi, h, :] . k[cu_k[b]+j, hk, :],  j < n
+ *     out = softmax(s) V,   lse = ln sum_j exp(s_j)     (natural log)
+ *   n = 0 gives out = 0 and lse = -inf.
+ *
+ * It runs as split-KV flash-decoding: each (sequence, KV head, KV chunk)
+ * block emits unnormalised (O, m, l) partials and a log-sum-exp merge
+ * produces the output (AstrAI commit log for csrc/kernels/gqa_decode_attn.cu,
+ * split-KV commit; magik.net "Wiring Split-K Dispatch into a Custom CUDA
+ * Attention Kernel", section "The Message").  The grid and the split count are
+ * fixed when the plan is made, from constants only, and the kernels read the
+ * exact lengths from device-side cu_seqlens, so a call makes no device-to-host
+ * copy, no allocation and no compilation and can be captured once in a CUDA
+ * graph and replayed while the lengths change (cudnn-frontend issue #552
+ * "frost(sdpa): THD execute host round-trip", section "Proposal to evaluate").
+ *
+ * Conventions for every entry point:
+ *  - Return value: 0 (ATTN_OK) or a negative ATTN_E_* code; attn_strerror()
+ *    names it.  On an error return nothing has been launched or changed.
+ *  - "device pointer" means memory of the CUDA device that was current when
+ *    the plan was made; the caller owns it and keeps it alive until the work
+ *    on the stream that uses it has finished.
+ *  - stream: a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  All device work of a call is ordered on that stream.
+ *  - Calls on one plan must not overlap on the GPU (the plan's scratch is
+ *    reused by every call); use one plan per concurrent stream.
+ *  - Thread safety: distinct plans may be used from distinct host threads.
+ */
+#ifndef VARLEN_GQA_H
+#define VARLEN_GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- errors */
+#define ATTN_OK 0
+#define ATTN_E_INVALID_ARG (-1)   /* a size or count out of range            */
+#define ATTN_E_UNSUPPORTED (-2)   /* e.g. head dim not in {64, 128}           */
+#define ATTN_E_NULL (-3)          /* a required pointer is NULL               */
+#define ATTN_E_ALIGNMENT (-4)     /* a pointer breaks the alignment contract  */
+#define ATTN_E_BAD_PLAN (-5)      /* unknown or destroyed plan handle         */
+#define ATTN_E_CUDA (-6)          /* a CUDA runtime / driver call failed      */
+#define ATTN_E_NOMEM (-7)         /* device allocation failed                 */
+#define ATTN_E_DEVICE (-8)        /* current device is not the plan's device  */
+#define ATTN_E_NO_DEVICE (-9)     /* no usable sm_100 device                  */
+
+/* Sticky device-side error bits, read by attn_check_error().  When a
+ * sequence trips one, none of its output rows are written. */
+#define ATTN_DEV_ERR_OFFSETS 0x1u      /* cu_q / cu_k negative or decreasing  */
+#define ATTN_DEV_ERR_Q_TOO_LONG 0x2u   /* Lq_b > max_q of the plan            */
+#define ATTN_DEV_ERR_K_TOO_LONG 0x4u   /* Lk_b > s_max of the plan            */
+#define ATTN_DEV_ERR_TIMEOUT 0x8u      /* a bounded pipeline wait gave up      */
+
+/* Kernel variants (attn_overrides.variant / attn_plan_desc.variant). */
+#define ATTN_VARIANT_AUTO 0
+#define ATTN_VARIANT_SIMT 1   /* CUDA-core path, any row count               */
+#define ATTN_VARIANT_MMA 2    /* TMA-fed tensor-core path, G*max_q <= 16      */
+
+/* How split partials are merged (attn_overrides.combine / attn_plan_desc.combine). */
+#define ATTN_COMBINE_AUTO 0
+#define ATTN_COMBINE_KERNEL 1  /* a second kernel merges every row                */
+#define ATTN_COMBINE_FUSED 2   /* the last block of each unit to finish merges it  */
+
+typedef struct attn_plan_s *attn_plan_t;   /* opaque */
+
+/*
+ * Explicit plan choices, for sweeps in tests and benchmarks (the magik.net
+ * post tunes its split count through an environment knob, section "Assumptions
+ * and Their Validity"; here it is an argument).  Zero in a field keeps the
+ * planner's own choice.
+ */
+typedef struct {
+    int nsplit;    /* KV chunks per (sequence, KV head); >= 1                  */
+    int block_n;   /* keys per pipeline tile: 64                                */
+    int variant;   /* ATTN_VARIANT_*                                            */
+    int stages;    /* pipeline depth of the tensor-core path: 2..8              */
+    int combine;   /* ATTN_COMBINE_*                                            */
+} attn_overrides;
+
+/* What the planner chose (attn_plan_info). */
+typedef struct {
+    int B_max, s_max, Hq, Hkv, D, max_q;
+    int G;                 /* Hq / Hkv                                          */
+    int variant;           /* ATTN_VARIANT_SIMT or ATTN_VARIANT_MMA             */
+    int nsplit;            /* KV chunks per (sequence, KV head)                  */
+    int chunk;             /* keys per chunk (multiple of block_n)               */
+    int block_n;           /* keys per tile                                      */
+    int stages;            /* pipeline stages (tensor-core path)                 */
+    int rows_per_block;    /* query rows (G * q tokens) one block handles        */
+    int row_tiles;         /* blocks along the row axis per KV head              */
+    int grid_x, grid_y, grid_z;   /* split-kernel grid: (nsplit, Hkv*row_tiles, B_max) */
+    int combine;           /* ATTN_COMBINE_KERNEL or ATTN_COMBINE_FUSED          */
+    int combine_blocks;    /* combine-kernel blocks (0 unless a combine kernel runs) */
+    int smem_bytes;        /* dynamic shared memory of the split kernel          */
+    int num_sms;           /* SM count of the plan's device                      */
+    size_t scratch_bytes;  /* device scratch the plan owns (partials)            */
+} attn_plan_desc;
+
+/*
+ * attn_plan -- size the grid and the split count once, from constants.
+ *
+ *   B_max  sequences per call (cu arrays hold B_max + 1 entries); >= 1
+ *   s_max  largest key length of any sequence; >= 1
+ *   Hq, Hkv  query / KV heads, Hq % Hkv == 0
+ *   D      head dimension, 64 or 128
+ *   max_q  largest query length of any sequence; 1 for decode; >= 1
+ *
+ * Source: plan-time grid from declared constants, cudnn-frontend issue #552,
+ * section "Proposal to evaluate"; split count that fills the device and falls
+ * back to a single direct-write pass when B*Hkv already saturates it, AstrAI
+ * commit log (split-KV commit); reject an unsupported head dim rather than run
+ * a silent fallback, AstrAI commit log (dispatch commit).
+ *
+ * Queries the current device's SM count, allocates the partials scratch and a
+ * device error word with cudaMalloc, and sets kernel attributes: call it
+ * outside stream capture.  The softmax scale is 1/sqrt(D) and the causal mask
+ * is aligned to each sequence's tail (a no-op when Lq_b = 1).  On success
+ * *out holds a new plan, owned by the caller until attn_destroy().
+ */
+int attn_plan(attn_plan_t *out, int B_max, int s_max, int Hq, int Hkv, int D,
+              int max_q);
+
+/* attn_plan with explicit choices; o may be NULL (same as attn_plan). */
+int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int Hkv, int D,
+                 int max_q, const attn_overrides *o);
+
+/* Fill *desc with the plan's choices.  Host only; never touches the GPU. */
+int attn_plan_info(attn_plan_t plan, attn_plan_desc *desc);
+
+/*
+ * attn_run -- one attention call, asynchronous on `stream`.
+ *
+ *   q      device, bf16 [T_q, Hq, D], packed and contiguous, 16-byte aligned
+ *   k, v   device, bf16 [T_kv, Hkv, D], packed and contiguous, 16-byte aligned;
+ *          readable for at least cu_k[B_max] tokens
+ *   cu_q, cu_k  device, int32, B_max + 1 entries each, 4-byte aligned:
+ *          cu[0] >= 0 and non-decreasing; sequence b owns tokens
+ *          [cu[b], cu[b+1]).  A batch smaller than B_max repeats its last
+ *          offset (zero-length sequences), the form a buffer sized for the
+ *          largest batch takes (TransformerEngine PR #24 "Build the attention
+ *          padding mask without host syncs", section Changes).
+ *   out    device, bf16 [T_q, Hq, D], 16-byte aligned
+ *   lse    device, fp32 [T_q, Hq] (natural log of the scaled scores), 4-byte
+ *          aligned
+ *
+ * Only rows covered by cu_q are written.  A sequence with Lk_b = 0 (or a
+ * query that sees no key) gets out = 0 and lse = -inf.  The lengths are read
+ * on the device; sequences that break the plan's bounds set a sticky bit for
+ * attn_check_error() and are left unwritten.
+ *
+ * The call launches one kernel (two with ATTN_COMBINE_KERNEL) and nothing
+ * else: no host sync, no
+ * device-to-host copy, no allocation, so it can be captured in a CUDA graph
+ * (the captured graph keeps the pointers; replay it with the same buffers,
+ * rewriting cu_q / cu_k and the tensors' contents in place).  Host-detectable
+ * errors (NULL or misaligned pointers, wrong device, bad plan) return a code
+ * and launch nothing.
+ */
+int attn_run(attn_plan_t plan, const void *q, const void *k, const void *v,
+             const int32_t *cu_q, const int32_t *cu_k, void *out, float *lse,
+             void *stream);
+
+/*
+ * attn_check_error -- synchronise `stream`, then read and clear the plan's
+ * sticky device error bits (ATTN_DEV_ERR_*) into *flags.  When a bit was set
+ * it also resets the plan's merge tickets, so the plan stays usable after a
+ * call that stopped early.  The only entry point that waits for the GPU; do
+ * not call it inside stream capture.
+ */
+int attn_check_error(attn_plan_t plan, void *stream, uint32_t *flags);
+
+/* Free the plan's device memory.  NULL or an unknown handle is ignored.  The
+ * caller must make sure no work that uses the plan is still pending. */
+void attn_destroy(attn_plan_t plan);
+
+/* Static message for an ATTN_* return code. */
+const char *attn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VARLEN_GQA_H */

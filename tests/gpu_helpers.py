@@ -1,0 +1,131 @@
+"""Shared helpers for the GPU tests: run the CUDA path through the C ABI and
+compare with the fp64 oracle on the same bytes."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import workloads as W
+from varlen_gqa_split_b200 import Plan
+
+# tolerances of the method's numerical contract: bf16 output and fp32 lse,
+# absolute, against the fp64 definition
+ATOL_OUT = 2e-2
+ATOL_LSE = 1e-3
+
+BF16_NAN_BITS = 0x7FC0
+
+
+def sentinel_out(T_q, Hq, D, device="cuda"):
+    """out buffer filled with a NaN bit pattern so untouched rows are visible."""
+    t = torch.full((T_q, Hq, D), BF16_NAN_BITS, dtype=torch.int16, device=device)
+    return t.view(torch.bfloat16)
+
+
+def sentinel_lse(T_q, Hq, device="cuda"):
+    return torch.full((T_q, Hq), float("nan"), dtype=torch.float32, device=device)
+
+
+def to_device(batch: W.Batch, device="cuda"):
+    q = batch.q.to(device).contiguous()
+    k = batch.k.to(device).contiguous()
+    v = batch.v.to(device).contiguous()
+    cu_q = torch.from_numpy(batch.cu_q).to(device)
+    cu_k = torch.from_numpy(batch.cu_k).to(device)
+    return q, k, v, cu_q, cu_k
+
+
+def run_gpu(plan: Plan, batch: W.Batch, extra_q_rows=0):
+    """Run on the GPU with sentinel-filled outputs; returns (out, lse) on host.
+
+    extra_q_rows: tail rows past cu_q[B_max] in the output buffers, which the
+    call must leave untouched."""
+    q, k, v, cu_q, cu_k = to_device(batch)
+    sh = batch.shape
+    T_q = q.shape[0] + extra_q_rows
+    if extra_q_rows:
+        q = torch.cat([q, torch.zeros(extra_q_rows, sh.Hq, sh.D, dtype=q.dtype, device=q.device)])
+    out = sentinel_out(T_q, sh.Hq, sh.D)
+    lse = sentinel_lse(T_q, sh.Hq)
+    plan.run(q, k, v, cu_q, cu_k, out, lse)
+    torch.cuda.synchronize()
+    assert plan.check_error() == 0
+    return out.cpu(), lse.cpu()
+
+
+def oracle_full(batch: W.Batch):
+    sh = batch.shape
+    return oracle.attention(W.bits(batch.q), W.bits(batch.k), W.bits(batch.v), batch.cu_q, batch.cu_k,
+                            B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D, causal=sh.causal)
+
+
+def covered_rows(batch: W.Batch) -> np.ndarray:
+    """Boolean mask over packed q tokens covered by cu_q."""
+    T = batch.q.shape[0]
+    m = np.zeros(T, dtype=bool)
+    m[: int(batch.cu_q[-1])] = True
+    return m
+
+
+def compare_full(out_gpu, lse_gpu, out_ref, lse_ref, covered, atol_out=ATOL_OUT, atol_lse=ATOL_LSE):
+    """Element-wise check of every covered row; rows not covered must keep
+    the NaN sentinel bit pattern.  Returns (max |out err|, max |lse err|)."""
+    o = out_gpu.float().numpy().astype(np.float64)
+    l = lse_gpu.numpy().astype(np.float64)
+    T = covered.shape[0]
+    oc, lc = o[:T][covered], l[:T][covered]
+    ro, rl = out_ref[:T][covered], lse_ref[:T][covered]
+    assert np.all(np.isfinite(oc)), "non-finite output in a covered row"
+    err_o = np.abs(oc - ro).max() if oc.size else 0.0
+    assert err_o <= atol_out, f"max |out - oracle| = {err_o}"
+    ninf_ref = np.isneginf(rl)
+    assert np.array_equal(np.isneginf(lc), ninf_ref), "-inf lse pattern differs from the oracle"
+    assert np.all(oc[ninf_ref] == 0.0), "rows with no visible key must be exactly 0"
+    fin = ~ninf_ref
+    err_l = np.abs(lc[fin] - rl[fin]).max() if fin.any() else 0.0
+    assert err_l <= atol_lse, f"max |lse - oracle| = {err_l}"
+    # untouched rows: bitwise sentinel
+    raw = out_gpu.view(torch.int16).numpy()
+    untouched = np.ones(raw.shape[0], dtype=bool)
+    untouched[:T] = ~covered
+    assert np.all(raw[untouched] == np.int16(BF16_NAN_BITS)), "a row outside cu_q was written"
+    assert np.all(np.isnan(l[untouched])), "an lse row outside cu_q was written"
+    return float(err_o), float(err_l)
+
+
+def sample_rows(batch: W.Batch, n, rng):
+    """(b, qi, h) triples: n random covered rows plus the first and last row of
+    every live sequence's last token for head 0 and the last head."""
+    sh = batch.shape
+    lens_q = np.diff(batch.cu_q)
+    live = np.nonzero(lens_q > 0)[0]
+    rows = set()
+    for b in live[: min(len(live), 64)]:
+        rows.add((int(b), int(lens_q[b]) - 1, 0))
+        rows.add((int(b), int(lens_q[b]) - 1, sh.Hq - 1))
+    while len(rows) < n + 2 * min(len(live), 64) and len(live):
+        b = int(rng.choice(live))
+        rows.add((b, int(rng.integers(0, lens_q[b])), int(rng.integers(0, sh.Hq))))
+    return np.array(sorted(rows), dtype=np.int64).reshape(-1, 3)
+
+
+def compare_rows(out_gpu, lse_gpu, batch: W.Batch, rows, atol_out=ATOL_OUT, atol_lse=ATOL_LSE):
+    sh = batch.shape
+    ro, rl = oracle.attention_rows(W.bits(batch.q), W.bits(batch.k), W.bits(batch.v), batch.cu_q,
+                                   batch.cu_k, rows, B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D,
+                                   causal=sh.causal)
+    tok = batch.cu_q[rows[:, 0]] + rows[:, 1]
+    o = out_gpu[tok, rows[:, 2]].float().numpy().astype(np.float64)
+    l = lse_gpu[tok, rows[:, 2]].numpy().astype(np.float64)
+    err_o = np.abs(o - ro).max()
+    assert err_o <= atol_out, f"max |out - oracle| = {err_o}"
+    assert np.array_equal(np.isneginf(l), np.isneginf(rl))
+    fin = np.isfinite(rl)
+    err_l = np.abs(l[fin] - rl[fin]).max() if fin.any() else 0.0
+    assert err_l <= atol_lse, f"max |lse - oracle| = {err_l}"
+    return float(err_o), float(err_l)
+
+
+def plan_for(shape: W.Shape, **kw) -> Plan:
+    return Plan(shape.B, shape.s_max, shape.Hq, shape.Hkv, shape.D, shape.max_q, **kw)

@@ -1,0 +1,285 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs (needs a B200).
+
+Every call goes through the C ABI (libvgqa.so via the ctypes binding).
+Tolerances: max-abs 2e-2 on the bf16 output, 1e-3 on the fp32 lse, -inf lse
+and zero output matched exactly, and cu_seqlens placement bit-exact (every
+covered row written, every other row keeps its NaN sentinel).
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from gpu_helpers import (ATOL_LSE, ATOL_OUT, compare_full, compare_rows, covered_rows, oracle_full,
+                         plan_for, run_gpu, sample_rows, sentinel_lse, sentinel_out, to_device)
+import varlen_gqa_split_b200 as vg
+
+pytestmark = pytest.mark.gpu
+
+SIMT, MMA = vg.ATTN_VARIANT_SIMT, vg.ATTN_VARIANT_MMA
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from varlen_gqa_split_b200 import build
+    build.build()
+    torch.cuda.init()
+
+
+def _gen_device(name):
+    return "cpu" if name == "tiny" else "cuda"
+
+
+# ------------------------------------------------------------ the five workloads
+
+@pytest.mark.parametrize("variant", [0, SIMT, MMA])
+@pytest.mark.parametrize("name", ["tiny", "long", "ragged"])
+def test_decode_workloads_full_parity(name, variant):
+    batch = W.workload(name, gen_device=_gen_device(name))
+    plan = plan_for(batch.shape, variant=variant)
+    out, lse = run_gpu(plan, batch, extra_q_rows=3)
+    ref_o, ref_l = oracle_full(batch)
+    cov = covered_rows(batch)
+    compare_full(out, lse, ref_o, ref_l, cov)
+
+
+@pytest.mark.parametrize("variant", [0, SIMT])
+def test_short_query_workload_full_parity(variant):
+    batch = W.workload("shortq", gen_device="cuda")
+    plan = plan_for(batch.shape, variant=variant)
+    out, lse = run_gpu(plan, batch, extra_q_rows=5)
+    ref_o, ref_l = oracle_full(batch)
+    compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
+
+
+def test_continuous_batching_one_graph_many_steps():
+    """One CUDA graph captured once (global capture mode: any host sync or
+    pageable copy inside attn_run would break the capture) and replayed for
+    100 steps while the lengths change in place; each step is checked against
+    the oracle on sampled rows."""
+    sh = W.SHAPES["continuous"]
+    steps = W.lengths("continuous", seed=0)
+    cap = max(int(lk.sum()) for _, lk in steps)
+    g = W.make_generator(0, "cuda")
+    k = W.bf16_normal((cap, sh.Hkv, sh.D), g, "cuda")
+    v = W.bf16_normal((cap, sh.Hkv, sh.D), g, "cuda")
+    qpool = W.bf16_normal((len(steps), sh.B, sh.Hq, sh.D), g, "cuda")
+    q = torch.empty(sh.B, sh.Hq, sh.D, dtype=torch.bfloat16, device="cuda")
+    cu_q = torch.from_numpy(W.cu_from_lengths(np.ones(sh.B, np.int64))).cuda()
+    cu_k = torch.zeros(sh.B + 1, dtype=torch.int32, device="cuda")
+    out = sentinel_out(sh.B, sh.Hq, sh.D)
+    lse = sentinel_lse(sh.B, sh.Hq)
+    plan = plan_for(sh)
+    cu_k.copy_(torch.from_numpy(W.cu_from_lengths(steps[0][1])))
+    q.copy_(qpool[0])
+    plan.run(q, k, v, cu_q, cu_k, out, lse)          # warm-up outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="global"):
+        plan.run(q, k, v, cu_q, cu_k, out, lse)
+    kb, vb = W.bits(k), W.bits(v)
+    rng = np.random.default_rng(0)
+    for s, (lq, lk) in enumerate(steps):
+        cu_k.copy_(torch.from_numpy(W.cu_from_lengths(lk)))
+        q.copy_(qpool[s])
+        graph.replay()
+        torch.cuda.synchronize()
+        batch = W.Batch(sh, q.cpu(), None, None, W.cu_from_lengths(lq), W.cu_from_lengths(lk), lq, lk)
+        rows = sample_rows(batch, 24, rng)
+        import oracle
+        ro, rl = oracle.attention_rows(W.bits(batch.q), kb, vb, batch.cu_q, batch.cu_k, rows, B=sh.B,
+                                       Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D)
+        oc = out.cpu()[rows[:, 0], rows[:, 2]].float().numpy()
+        lc = lse.cpu()[rows[:, 0], rows[:, 2]].numpy()
+        assert np.abs(oc - ro).max() <= ATOL_OUT, f"step {s}"
+        assert np.abs(lc - rl).max() <= ATOL_LSE, f"step {s}"
+    assert plan.check_error() == 0
+    del graph
+
+
+# ------------------------------------------------------------ split-count invariance
+
+@pytest.mark.parametrize("combine", [vg.ATTN_COMBINE_FUSED, vg.ATTN_COMBINE_KERNEL])
+@pytest.mark.parametrize("variant", [SIMT, MMA])
+def test_nsplit_invariance(variant, combine):
+    sh = W.Shape("mid", B=4, Hq=64, Hkv=8, D=128, max_q=1, s_max=4096)
+    batch = W.make_batch(sh, [1, 1, 1, 1], [4096, 1000, 77, 0], seed=3, gen_device="cuda")
+    ref_o, ref_l = oracle_full(batch)
+    cov = covered_rows(batch)
+    outs = []
+    for ns in (1, 2, 3, 8, 32, 64):
+        plan = plan_for(sh, variant=variant, nsplit=ns, combine=combine)
+        assert plan.info["nsplit"] == ns
+        assert plan.info["combine"] == (0 if ns == 1 else combine)
+        out, lse = run_gpu(plan, batch)
+        compare_full(out, lse, ref_o, ref_l, cov)
+        outs.append(out.float().numpy())
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= 2 * ATOL_OUT
+
+
+def test_variants_agree():
+    batch = W.workload("ragged", gen_device="cuda")
+    a, la = run_gpu(plan_for(batch.shape, variant=SIMT), batch)
+    b, lb = run_gpu(plan_for(batch.shape, variant=MMA), batch)
+    cov = covered_rows(batch)
+    fa, fb = a.float().numpy()[cov], b.float().numpy()[cov]
+    assert np.abs(fa - fb).max() <= 2 * ATOL_OUT
+    l1, l2 = la.numpy()[cov], lb.numpy()[cov]
+    fin = np.isfinite(l1)
+    assert np.array_equal(fin, np.isfinite(l2))
+    assert np.abs(l1[fin] - l2[fin]).max() <= 2 * ATOL_LSE
+
+
+@pytest.mark.parametrize("combine", [vg.ATTN_COMBINE_FUSED, vg.ATTN_COMBINE_KERNEL])
+def test_repeat_runs_bitwise_equal(combine):
+    # a fixed plan is deterministic: the merge order does not depend on which
+    # block of a unit finishes last
+    batch = W.workload("long", gen_device="cuda")
+    plan = plan_for(batch.shape, combine=combine)
+    runs = [run_gpu(plan, batch) for _ in range(3)]
+    for o, l in runs[1:]:
+        assert torch.equal(o.view(torch.int16), runs[0][0].view(torch.int16))
+        assert torch.equal(l.view(torch.int32), runs[0][1].view(torch.int32))
+
+
+# ------------------------------------------------------------ placement and edge cases
+
+def _packed_cases(B, values):
+    lq, lk = [], []
+    for lens_q in itertools.product(values, repeat=B):
+        for lens_k in itertools.product(values, repeat=B):
+            lq.extend(lens_q)
+            lk.extend(lens_k)
+    return lq, lk
+
+
+@pytest.mark.parametrize("variant", [SIMT, MMA])
+def test_exhaustive_small_lengths_placement(variant):
+    """Every (Lq, Lk) combination with lengths in [0, 4] for 3 sequences (the
+    exhaustive method of TransformerEngine PR #24, section Equivalence), packed
+    into one batch and padded with zero-length sequences to B_max; causal tail
+    alignment with Lq > Lk included."""
+    lq, lk = _packed_cases(3, range(5))
+    B_max = len(lq) + 7
+    sh = W.Shape("placement", B=B_max, Hq=4, Hkv=1, D=64, max_q=4, s_max=4)
+    batch = W.make_batch(sh, lq, lk, seed=11, gen_device="cuda")
+    plan = plan_for(sh, variant=variant)
+    out, lse = run_gpu(plan, batch, extra_q_rows=2)
+    ref_o, ref_l = oracle_full(batch)
+    compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
+
+
+@pytest.mark.parametrize("combine", [vg.ATTN_COMBINE_FUSED, vg.ATTN_COMBINE_KERNEL])
+@pytest.mark.parametrize("variant,nsplit", [(SIMT, 1), (SIMT, 3), (MMA, 1), (MMA, 2), (MMA, 5)])
+def test_ragged_multi_tile_placement(variant, nsplit, combine):
+    """Lengths spanning several 64-key tiles and chunks, short sequences whose
+    tile starts before the buffer (negative TMA coordinates), Lq up to 2."""
+    rng = np.random.default_rng(5 + nsplit)
+    B = 40
+    lq = rng.integers(0, 3, B)
+    lk = rng.integers(0, 330, B)
+    lk[:3] = [1, 63, 64]
+    lk[3:6] = [65, 0, 129]
+    sh = W.Shape("ragged_mt", B=B + 2, Hq=16, Hkv=2, D=128, max_q=2, s_max=330)
+    batch = W.make_batch(sh, lq, lk, seed=7, gen_device="cuda")
+    plan = plan_for(sh, variant=variant, nsplit=nsplit, combine=combine)
+    out, lse = run_gpu(plan, batch, extra_q_rows=1)
+    ref_o, ref_l = oracle_full(batch)
+    compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
+
+
+@pytest.mark.parametrize("variant", [SIMT, MMA])
+def test_single_key_returns_v_exactly(variant):
+    sh = W.Shape("one", B=5, Hq=8, Hkv=2, D=128, max_q=1, s_max=64)
+    batch = W.make_batch(sh, [1] * 5, [1] * 5, seed=2, gen_device="cuda")
+    plan = plan_for(sh, variant=variant)
+    out, lse = run_gpu(plan, batch)
+    G = sh.Hq // sh.Hkv
+    want = batch.v.cpu().repeat_interleave(G, dim=1)
+    assert torch.equal(out.view(torch.int16), want.view(torch.int16))
+
+
+@pytest.mark.parametrize("variant", [SIMT, MMA])
+def test_large_magnitude_scores(variant):
+    sh = W.Shape("big", B=2, Hq=8, Hkv=1, D=128, max_q=1, s_max=2048)
+    batch = W.make_batch(sh, [1, 1], [2048, 513], seed=4, gen_device="cuda")
+    batch.q = (batch.q.float() * 30).to(torch.bfloat16)
+    plan = plan_for(sh, variant=variant, nsplit=4)
+    out, lse = run_gpu(plan, batch)
+    ref_o, ref_l = oracle_full(batch)
+    compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
+
+
+def test_plan_choices_follow_the_split_rule():
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    long_plan = plan_for(W.SHAPES["long"])
+    assert long_plan.info["nsplit"] > 1 and long_plan.info["variant"] == MMA
+    assert long_plan.info["grid_x"] * long_plan.info["grid_y"] >= sms
+    ragged_plan = plan_for(W.SHAPES["ragged"])
+    assert ragged_plan.info["nsplit"] == 1          # B * Hkv = 512 blocks already fill the SMs
+    assert ragged_plan.info["scratch_bytes"] <= 1024
+    sq = plan_for(W.SHAPES["shortq"])
+    assert sq.info["variant"] == SIMT
+
+
+# ------------------------------------------------------------ errors
+
+def test_device_side_errors_are_flagged_and_rows_untouched():
+    sh = W.Shape("err", B=3, Hq=8, Hkv=2, D=128, max_q=1, s_max=64)
+    plan = plan_for(sh)
+    g = W.make_generator(1, "cuda")
+    T = 200
+    q = W.bf16_normal((T, sh.Hq, sh.D), g, "cuda")
+    k = W.bf16_normal((T, sh.Hkv, sh.D), g, "cuda")
+    v = W.bf16_normal((T, sh.Hkv, sh.D), g, "cuda")
+    cases = [
+        ([0, 1, 2, 3], [0, 10, 75, 80], vg.ATTN_DEV_ERR_K_TOO_LONG, {1}),     # Lk = 65 > s_max
+        ([0, 1, 3, 4], [0, 10, 20, 30], vg.ATTN_DEV_ERR_Q_TOO_LONG, {1}),     # Lq = 2 > max_q
+        ([0, 1, 2, 3], [0, 10, 5, 30], vg.ATTN_DEV_ERR_OFFSETS, {1}),         # decreasing cu_k
+    ]
+    for cq, ck, bit, bad in cases:
+        out = sentinel_out(T, sh.Hq, sh.D)
+        lse = sentinel_lse(T, sh.Hq)
+        cu_q = torch.tensor(cq, dtype=torch.int32, device="cuda")
+        cu_k = torch.tensor(ck, dtype=torch.int32, device="cuda")
+        plan.run(q, k, v, cu_q, cu_k, out, lse)
+        flags = plan.check_error()
+        assert flags & bit, (flags, bit)
+        assert plan.check_error() == 0                       # read-and-clear
+        raw = out.view(torch.int16).cpu()
+        for b in range(3):
+            rows = range(cq[b], cq[b + 1])
+            for r in rows:
+                written = not bool(torch.all(raw[r] == np.int16(0x7FC0)))
+                assert written == (b not in bad), (cq, ck, b)
+
+
+def test_host_side_errors_launch_nothing():
+    import ctypes
+    L = vg.lib()
+    sh = W.Shape("h", B=1, Hq=4, Hkv=1, D=64, max_q=1, s_max=64)
+    plan = plan_for(sh)
+    q = torch.zeros(4, 4, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(4, 1, 64, dtype=torch.bfloat16, device="cuda")
+    cu = torch.tensor([0, 1], dtype=torch.int32, device="cuda")
+    out = torch.zeros_like(q)
+    lse = torch.zeros(4, 4, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    h = plan.handle
+    assert L.attn_run(h, q.data_ptr() + 2, k.data_ptr(), k.data_ptr(), cu.data_ptr(), cu.data_ptr(),
+                      out.data_ptr(), lse.data_ptr(), s) == -4
+    assert L.attn_run(h, None, k.data_ptr(), k.data_ptr(), cu.data_ptr(), cu.data_ptr(),
+                      out.data_ptr(), lse.data_ptr(), s) == -3
+    with pytest.raises(vg.AttnError):
+        vg.Plan(1, 64, 4, 1, 96, 1)                         # unsupported head dim
+    with pytest.raises(vg.AttnError):
+        vg.Plan(1, 64, 64, 8, 128, 4, variant=MMA)         # 32 rows > tensor-core path limit
+    handle = plan.handle
+    plan.close()
+    assert L.attn_run(handle, q.data_ptr(), k.data_ptr(), k.data_ptr(), cu.data_ptr(), cu.data_ptr(),
+                      out.data_ptr(), lse.data_ptr(), s) == -5
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)

@@ -1,0 +1,183 @@
+"""ctypes binding of libvgqa (include/varlen_gqa.h): argument marshalling only.
+
+Every step of the attention runs in the library's CUDA kernels; this module
+checks dtypes, shapes and devices of torch tensors, passes their device
+pointers and the current CUDA stream, and turns ATTN_* codes into exceptions.
+There is no fallback: if the library is missing or no sm_100 device is
+present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libvgqa.so")
+
+ATTN_OK = 0
+ATTN_VARIANT_AUTO, ATTN_VARIANT_SIMT, ATTN_VARIANT_MMA = 0, 1, 2
+ATTN_COMBINE_AUTO, ATTN_COMBINE_KERNEL, ATTN_COMBINE_FUSED = 0, 1, 2
+ATTN_DEV_ERR_OFFSETS = 0x1
+ATTN_DEV_ERR_Q_TOO_LONG = 0x2
+ATTN_DEV_ERR_K_TOO_LONG = 0x4
+ATTN_DEV_ERR_TIMEOUT = 0x8
+
+EXPORTED = ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_check_error",
+            "attn_destroy", "attn_strerror")
+
+
+class Overrides(ctypes.Structure):
+    _fields_ = [("nsplit", ctypes.c_int), ("block_n", ctypes.c_int), ("variant", ctypes.c_int),
+                ("stages", ctypes.c_int), ("combine", ctypes.c_int)]
+
+
+class PlanDesc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "B_max", "s_max", "Hq", "Hkv", "D", "max_q", "G", "variant", "nsplit", "chunk", "block_n",
+        "stages", "rows_per_block", "row_tiles", "grid_x", "grid_y", "grid_z", "combine", "combine_blocks",
+        "smem_bytes", "num_sms")] + [("scratch_bytes", ctypes.c_size_t)]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (code {code})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvgqa.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libvgqa.so not built ({LIB_PATH}); run "
+                               "`python -m varlen_gqa_split_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, i32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+        L.attn_plan.argtypes = [ctypes.POINTER(vp), i, i, i, i, i, i]
+        L.attn_plan.restype = i
+        L.attn_plan_ex.argtypes = [ctypes.POINTER(vp), i, i, i, i, i, i, ctypes.POINTER(Overrides)]
+        L.attn_plan_ex.restype = i
+        L.attn_plan_info.argtypes = [vp, ctypes.POINTER(PlanDesc)]
+        L.attn_plan_info.restype = i
+        L.attn_run.argtypes = [vp, vp, vp, vp, i32p, i32p, vp, vp, vp]
+        L.attn_run.restype = i
+        L.attn_check_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.attn_check_error.restype = i
+        L.attn_destroy.argtypes = [vp]
+        L.attn_destroy.restype = None
+        L.attn_strerror.argtypes = [i]
+        L.attn_strerror.restype = ctypes.c_char_p
+        _lib = L
+        return L
+
+
+def strerror(code: int) -> str:
+    return lib().attn_strerror(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != ATTN_OK:
+        raise AttnError(code, where)
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Plan:
+    """A plan: launch shape, split count and scratch fixed from constants.
+
+    Plan(B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
+    stages=0, combine=0) -- the keyword choices override the planner (0 = its own)."""
+
+    def __init__(self, B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
+                 stages=0, combine=0):
+        L = lib()
+        h = ctypes.c_void_p()
+        if nsplit or block_n or variant or stages or combine:
+            o = Overrides(int(nsplit), int(block_n), int(variant), int(stages), int(combine))
+            rc = L.attn_plan_ex(ctypes.byref(h), int(B_max), int(s_max), int(Hq), int(Hkv), int(D),
+                                int(max_q), ctypes.byref(o))
+        else:
+            rc = L.attn_plan(ctypes.byref(h), int(B_max), int(s_max), int(Hq), int(Hkv), int(D),
+                             int(max_q))
+        _check(rc, "attn_plan")
+        self._h = h
+        self.device = torch.cuda.current_device()
+        self.info = self._info()
+
+    def _info(self) -> dict:
+        d = PlanDesc()
+        _check(lib().attn_plan_info(self._h, ctypes.byref(d)), "attn_plan_info")
+        return {name: getattr(d, name) for name, _ in PlanDesc._fields_}
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        return self._h
+
+    def run(self, q, k, v, cu_q, cu_k, out=None, lse=None, stream=None):
+        """out, lse = plan.run(q, k, v, cu_q, cu_k[, out, lse, stream]).
+
+        q [T_q, Hq, D], k / v [T_kv, Hkv, D] bf16 contiguous CUDA tensors;
+        cu_q / cu_k int32 CUDA tensors with B_max + 1 entries; out / lse are
+        allocated when not given (pass them for graph capture)."""
+        if self._h is None:
+            raise AttnError(-5, "attn_run")
+        i = self.info
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+                raise TypeError(f"{name} must be a contiguous bf16 CUDA tensor")
+        if q.dim() != 3 or q.shape[1:] != (i["Hq"], i["D"]):
+            raise ValueError(f"q must be [T_q, {i['Hq']}, {i['D']}]")
+        for name, t in (("k", k), ("v", v)):
+            if t.dim() != 3 or t.shape[1:] != (i["Hkv"], i["D"]):
+                raise ValueError(f"{name} must be [T_kv, {i['Hkv']}, {i['D']}]")
+        for name, t in (("cu_q", cu_q), ("cu_k", cu_k)):
+            if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.numel() != i["B_max"] + 1:
+                raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of B_max+1 entries")
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(q.shape[0], i["Hq"], dtype=torch.float32, device=q.device)
+        if out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous():
+            raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+        if lse.dtype != torch.float32 or lse.shape != (q.shape[0], i["Hq"]) or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous fp32 tensor [T_q, Hq]")
+        rc = lib().attn_run(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_q.data_ptr(),
+                            cu_k.data_ptr(), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
+        _check(rc, "attn_run")
+        return out, lse
+
+    def check_error(self, stream=None) -> int:
+        """Synchronise, then read and clear the sticky device error bits."""
+        f = ctypes.c_uint32(0)
+        _check(lib().attn_check_error(self._h, _stream_ptr(stream), ctypes.byref(f)), "attn_check_error")
+        return int(f.value)
+
+    def close(self):
+        if self._h is not None:
+            lib().attn_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()

@@ -1,0 +1,358 @@
+// api.cpp -- the C ABI of libvgqa (declared in include/varlen_gqa.h).
+//
+// attn_plan fixes everything that shapes the launch -- kernel variant, split
+// count, chunk length, grid, scratch -- from constants (B_max, s_max, head
+// counts, head dim, max_q, the device's SM count), so attn_run only fills a
+// parameter block, encodes two TMA descriptors on the host and launches: no
+// device-to-host copy, no allocation, no compilation (cudnn-frontend issue
+// #552 "frost(sdpa): THD execute host round-trip", sections Context and
+// Proposal to evaluate).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+#include <unordered_set>
+
+#include "../../include/varlen_gqa.h"
+#include "kernels.h"
+#include "params.h"
+
+#define ATTN_EXPORT extern "C" __attribute__((visibility("default")))
+
+using namespace vgqa;
+
+struct attn_plan_s {
+    attn_plan_desc d;
+    int device;
+    int NT;                    // tensor-core path: row fragments of 8
+    float scale_log2;
+    void *scratch;             // one allocation: error word, partials
+    uint32_t *err;
+    uint32_t *ticket;          // fused-merge arrival counters
+    size_t ticket_bytes;
+    float *o_part;
+    float2 *ml_part;
+};
+
+namespace {
+
+std::mutex g_mu;
+std::unordered_set<attn_plan_s *> g_plans;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool live(attn_plan_s *p) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_plans.count(p) != 0;
+}
+
+int get_encoder() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode) return ATTN_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return ATTN_E_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return ATTN_OK;
+}
+
+// [T, Hkv, D] bf16, box = 64 elements x 1 head x block_n tokens, 128-byte
+// swizzle.  The token extent is left open (2^31 - 1): every load the kernel
+// issues ends at or before its sequence's last key (cu_k[b+1] - 1), so the
+// real buffer length never enters.
+int encode_kv_map(CUtensorMap *map, const void *base, int Hkv, int D, int block_n) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)0x7fffffff};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)block_n};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void *ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+}  // namespace
+
+ATTN_EXPORT const char *attn_strerror(int code) {
+    switch (code) {
+    case ATTN_OK: return "success";
+    case ATTN_E_INVALID_ARG: return "invalid argument (size or count out of range)";
+    case ATTN_E_UNSUPPORTED: return "unsupported configuration (head dim must be 64 or 128)";
+    case ATTN_E_NULL: return "a required pointer is NULL";
+    case ATTN_E_ALIGNMENT: return "a pointer breaks the alignment contract (16 B tensors, 4 B cu/lse)";
+    case ATTN_E_BAD_PLAN: return "unknown or destroyed plan";
+    case ATTN_E_CUDA: return "a CUDA call failed";
+    case ATTN_E_NOMEM: return "device allocation failed";
+    case ATTN_E_DEVICE: return "current device differs from the plan's device";
+    case ATTN_E_NO_DEVICE: return "no usable sm_100 device";
+    default: return "unknown error code";
+    }
+}
+
+ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int Hkv, int D, int max_q,
+                             const attn_overrides *o) {
+    if (!out) return ATTN_E_NULL;
+    *out = nullptr;
+    if (B_max < 1 || B_max > 65535 || s_max < 1 || s_max > (1 << 30) || Hq < 1 || Hkv < 1 ||
+        Hq % Hkv != 0 || max_q < 1 || max_q > 65536)
+        return ATTN_E_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_E_UNSUPPORTED;
+    const long long rows = (long long)(Hq / Hkv) * max_q;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_E_NO_DEVICE;
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return ATTN_E_NO_DEVICE;
+    if (major != 10) return ATTN_E_NO_DEVICE;
+
+    attn_plan_desc d{};
+    d.B_max = B_max;
+    d.s_max = s_max;
+    d.Hq = Hq;
+    d.Hkv = Hkv;
+    d.D = D;
+    d.max_q = max_q;
+    d.G = Hq / Hkv;
+    d.num_sms = sms;
+
+    int variant = o && o->variant ? o->variant : (rows <= 16 ? ATTN_VARIANT_MMA : ATTN_VARIANT_SIMT);
+    if (variant != ATTN_VARIANT_MMA && variant != ATTN_VARIANT_SIMT) return ATTN_E_INVALID_ARG;
+    if (variant == ATTN_VARIANT_MMA && rows > 16) return ATTN_E_UNSUPPORTED;
+    if (o && o->block_n && o->block_n != 64) return ATTN_E_UNSUPPORTED;
+    d.variant = variant;
+
+    int NT = 1;
+    int per_sm = 1;
+    if (variant == ATTN_VARIANT_MMA) {
+        NT = rows <= 8 ? 1 : 2;
+        d.block_n = mma_block_n();
+        d.stages = o && o->stages ? o->stages : (D == 128 ? 3 : 4);
+        if (d.stages < 2 || d.stages > 8) return ATTN_E_INVALID_ARG;
+        d.rows_per_block = 8 * NT;
+        d.row_tiles = 1;
+        d.smem_bytes = (int)mma_smem_bytes(D, NT, d.stages);
+        if (mma_prepare(D, NT, d.stages) != cudaSuccess) return ATTN_E_CUDA;
+    } else {
+        d.block_n = kSimtBlockN;
+        d.stages = 2;
+        d.rows_per_block = kSimtRowsPerBlock;
+        d.row_tiles = (int)((rows + kSimtRowsPerBlock - 1) / kSimtRowsPerBlock);
+        d.smem_bytes = (int)simt_smem_bytes(D);
+        if (simt_prepare(D) != cudaSuccess) return ATTN_E_CUDA;
+    }
+    if ((long long)Hkv * d.row_tiles > 65535) return ATTN_E_INVALID_ARG;
+    {
+        // resident blocks per SM, from shared memory (the binding limit here)
+        int smem_sm = 0;
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        per_sm = std::max(1, smem_sm / (d.smem_bytes + 1024));
+        per_sm = std::min(per_sm, 4);
+    }
+
+    // Split count: fill the device (about per_sm blocks per SM), capped by the
+    // tile count; fall back to one direct-write pass when the (sequence, KV
+    // head, row tile) units alone already fill it (AstrAI commit log,
+    // split-KV commit).
+    const long long units = (long long)B_max * Hkv * d.row_tiles;
+    const long long target = (long long)sms * per_sm;
+    const int tiles_max = (s_max + d.block_n - 1) / d.block_n;
+    long long ns;
+    if (o && o->nsplit) {
+        if (o->nsplit < 1) return ATTN_E_INVALID_ARG;
+        ns = o->nsplit;
+    } else if (units >= target) {
+        ns = 1;
+    } else {
+        ns = (target + units - 1) / units;
+    }
+    ns = std::max(1LL, std::min<long long>(ns, std::min(tiles_max, 1024)));
+    const int tiles_per_chunk = (int)((tiles_max + ns - 1) / ns);
+    d.chunk = tiles_per_chunk * d.block_n;
+    d.nsplit = (s_max + d.chunk - 1) / d.chunk;
+    d.grid_x = d.nsplit;
+    d.grid_y = Hkv * d.row_tiles;
+    d.grid_z = B_max;
+
+    // how split partials are merged: by the last block of each unit (one
+    // launch per call) when its shared memory holds the merge tables, else by
+    // a second kernel
+    int combine = 0;
+    if (d.nsplit > 1) {
+        const size_t need = (size_t)d.rows_per_block * (d.nsplit + 1) * 8;
+        const size_t cap = variant == ATTN_VARIANT_MMA ? mma_merge_capacity(D, d.stages) : simt_merge_capacity(D);
+        const int want = o && o->combine ? o->combine : ATTN_COMBINE_FUSED;
+        if (want != ATTN_COMBINE_KERNEL && want != ATTN_COMBINE_FUSED) return ATTN_E_INVALID_ARG;
+        combine = (want == ATTN_COMBINE_FUSED && need <= cap) ? ATTN_COMBINE_FUSED : ATTN_COMBINE_KERNEL;
+    }
+    d.combine = combine;
+
+    // scratch: error word, merge tickets, then (nsplit > 1) O partials and
+    // (m, l) partials
+    const size_t n_part = d.nsplit > 1 ? (size_t)B_max * max_q * Hq * d.nsplit : 0;
+    const size_t n_ticket = combine == ATTN_COMBINE_FUSED ? (size_t)B_max * Hkv * d.row_tiles : 0;
+    const size_t off_t = 256;
+    const size_t off_o = align_up(off_t + n_ticket * sizeof(uint32_t), 256);
+    const size_t off_ml = align_up(off_o + n_part * D * sizeof(float), 256);
+    const size_t total = align_up(off_ml + n_part * sizeof(float2), 256);
+    d.scratch_bytes = total;
+
+    attn_plan_s *p = new (std::nothrow) attn_plan_s{};
+    if (!p) return ATTN_E_NOMEM;
+    p->d = d;
+    p->device = dev;
+    p->NT = NT;
+    p->scale_log2 = (float)((1.0 / std::sqrt((double)D)) * 1.4426950408889634);
+    if (cudaMalloc(&p->scratch, total) != cudaSuccess) {
+        cudaGetLastError();
+        delete p;
+        return ATTN_E_NOMEM;
+    }
+    p->err = static_cast<uint32_t *>(p->scratch);
+    p->ticket = n_ticket ? reinterpret_cast<uint32_t *>(static_cast<char *>(p->scratch) + off_t) : nullptr;
+    p->ticket_bytes = n_ticket * sizeof(uint32_t);
+    p->o_part = n_part ? reinterpret_cast<float *>(static_cast<char *>(p->scratch) + off_o) : nullptr;
+    p->ml_part = n_part ? reinterpret_cast<float2 *>(static_cast<char *>(p->scratch) + off_ml) : nullptr;
+    if (cudaMemset(p->scratch, 0, off_o) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(p->scratch);
+        delete p;
+        return ATTN_E_CUDA;
+    }
+    d.combine_blocks = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_plans.insert(p);
+    }
+    if (variant == ATTN_VARIANT_MMA) {
+        int rc = get_encoder();
+        if (rc != ATTN_OK) {
+            attn_destroy(p);
+            return rc;
+        }
+    }
+    if (combine == ATTN_COMBINE_KERNEL) {
+        Params tmp{};
+        tmp.B_max = B_max;
+        tmp.max_q = max_q;
+        tmp.Hq = Hq;
+        p->d.combine_blocks = combine_blocks(tmp);
+    }
+    if (std::getenv("VGQA_LOG"))
+        std::fprintf(stderr,
+                     "[vgqa] plan B_max=%d s_max=%d Hq=%d Hkv=%d D=%d max_q=%d: variant=%d nsplit=%d "
+                     "chunk=%d grid=(%d,%d,%d) smem=%d stages=%d per_sm=%d combine=%d scratch=%zu\n",
+                     B_max, s_max, Hq, Hkv, D, max_q, p->d.variant, p->d.nsplit, p->d.chunk, p->d.grid_x,
+                     p->d.grid_y, p->d.grid_z, p->d.smem_bytes, p->d.stages, per_sm, p->d.combine,
+                     p->d.scratch_bytes);
+    *out = p;
+    return ATTN_OK;
+}
+
+ATTN_EXPORT int attn_plan(attn_plan_t *out, int B_max, int s_max, int Hq, int Hkv, int D, int max_q) {
+    return attn_plan_ex(out, B_max, s_max, Hq, Hkv, D, max_q, nullptr);
+}
+
+ATTN_EXPORT int attn_plan_info(attn_plan_t plan, attn_plan_desc *desc) {
+    if (!desc) return ATTN_E_NULL;
+    if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
+    *desc = plan->d;
+    return ATTN_OK;
+}
+
+ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const void *v, const int32_t *cu_q,
+                         const int32_t *cu_k, void *out, float *lse, void *stream) {
+    if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
+    if (!q || !k || !v || !cu_q || !cu_k || !out || !lse) return ATTN_E_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+        !aligned(cu_q, 4) || !aligned(cu_k, 4))
+        return ATTN_E_ALIGNMENT;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_E_CUDA;
+    if (dev != plan->device) return ATTN_E_DEVICE;
+
+    const attn_plan_desc &d = plan->d;
+    Params p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    p.o_part = plan->o_part;
+    p.ml_part = plan->ml_part;
+    p.err = plan->err;
+    p.B_max = d.B_max;
+    p.s_max = d.s_max;
+    p.Hq = d.Hq;
+    p.Hkv = d.Hkv;
+    p.D = d.D;
+    p.max_q = d.max_q;
+    p.G = d.G;
+    p.nsplit = d.nsplit;
+    p.chunk = d.chunk;
+    p.rows_per_block = d.rows_per_block;
+    p.row_tiles = d.row_tiles;
+    p.scale_log2 = plan->scale_log2;
+    p.ticket = plan->ticket;
+    p.fused = d.combine == ATTN_COMBINE_FUSED;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid(d.grid_x, d.grid_y, d.grid_z);
+    cudaError_t e;
+    if (d.variant == ATTN_VARIANT_MMA) {
+        CUtensorMap tm_k, tm_v;
+        if (encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n) != ATTN_OK ||
+            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n) != ATTN_OK)
+            return ATTN_E_CUDA;
+        e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, grid, s);
+    } else {
+        e = launch_split_simt(p, grid, s);
+    }
+    if (e != cudaSuccess) return ATTN_E_CUDA;
+    if (d.combine == ATTN_COMBINE_KERNEL) {
+        e = launch_combine(p, s);
+        if (e != cudaSuccess) return ATTN_E_CUDA;
+    }
+    return ATTN_OK;
+}
+
+ATTN_EXPORT int attn_check_error(attn_plan_t plan, void *stream, uint32_t *flags) {
+    if (!flags) return ATTN_E_NULL;
+    *flags = 0;
+    if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t h = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_E_CUDA;
+    if (cudaMemcpy(&h, plan->err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_E_CUDA;
+    if (cudaMemset(plan->err, 0, sizeof(uint32_t)) != cudaSuccess) return ATTN_E_CUDA;
+    // a call that stopped early may have left merge tickets part-counted
+    if (h && plan->ticket_bytes && cudaMemset(plan->ticket, 0, plan->ticket_bytes) != cudaSuccess)
+        return ATTN_E_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_E_CUDA;
+    *flags = h;
+    return ATTN_OK;
+}
+
+ATTN_EXPORT void attn_destroy(attn_plan_t plan) {
+    if (!plan) return;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_plans.erase(plan)) return;
+    }
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != plan->device) cudaSetDevice(plan->device);
+    cudaFree(plan->scratch);
+    if (prev >= 0 && prev != plan->device) cudaSetDevice(prev);
+    delete plan;
+}

@@ -1,0 +1,33 @@
+// kernels.h -- host-side launchers of libvgqa's kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace vgqa {
+
+struct Params;
+
+// CUDA-core split kernel (any row count), 16 query rows per block
+size_t simt_smem_bytes(int D);
+size_t simt_merge_capacity(int D);
+cudaError_t simt_prepare(int D);
+cudaError_t launch_split_simt(const Params &p, dim3 grid, cudaStream_t stream);
+constexpr int kSimtRowsPerBlock = 16;
+constexpr int kSimtBlockN = 64;
+
+// TMA-fed tensor-core split kernel, NT = ceil(G * max_q / 8) in {1, 2}
+size_t mma_smem_bytes(int D, int NT, int stages);
+size_t mma_merge_capacity(int D, int stages);
+int mma_block_n();
+int mma_threads();
+cudaError_t mma_prepare(int D, int NT, int stages);
+cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUtensorMap &tm_v, int NT,
+                             int stages, dim3 grid, cudaStream_t stream);
+
+// log-sum-exp merge of the split partials
+int combine_blocks(const Params &p);
+cudaError_t launch_combine(const Params &p, cudaStream_t stream);
+
+}  // namespace vgqa

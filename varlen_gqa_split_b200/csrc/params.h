@@ -1,0 +1,32 @@
+// params.h -- launch parameter block shared by host code and kernels (internal).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace vgqa {
+
+// Everything a split / combine launch needs.  Passed by value.
+struct Params {
+    const __nv_bfloat16 *q;    // [T_q, Hq, D]
+    const __nv_bfloat16 *k;    // [T_kv, Hkv, D]
+    const __nv_bfloat16 *v;    // [T_kv, Hkv, D]
+    const int32_t *cu_q;       // [B_max + 1]
+    const int32_t *cu_k;       // [B_max + 1]
+    __nv_bfloat16 *out;        // [T_q, Hq, D]
+    float *lse;                // [T_q, Hq]
+    float *o_part;             // [B_max, max_q, Hq, nsplit, D]  (nsplit > 1)
+    float2 *ml_part;           // [B_max, max_q, Hq, nsplit]     (m, l) base-2
+    uint32_t *err;             // sticky ATTN_DEV_ERR_* bits
+    uint32_t *ticket;          // [B_max * Hkv * row_tiles] arrival counters (fused merge)
+    int B_max, s_max, Hq, Hkv, D, max_q, G;
+    int nsplit;                // chunks per (sequence, KV head)
+    int chunk;                 // keys per chunk
+    int rows_per_block;        // query rows (G * tokens) per block
+    int row_tiles;             // row blocks per KV head
+    float scale_log2;          // (1/sqrt(D)) * log2(e)
+    int fused;                 // nsplit > 1: the last block of a unit merges it
+};
+
+}  // namespace vgqa
