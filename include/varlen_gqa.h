@@ -55,6 +55,8 @@ extern "C" {
 #define ATTN_E_NOMEM (-7)         /* device allocation failed                 */
 #define ATTN_E_DEVICE (-8)        /* current device is not the plan's device  */
 #define ATTN_E_NO_DEVICE (-9)     /* no usable sm_100 device                  */
+#define ATTN_E_SCRATCH_LIMIT (-10) /* attn_run_noalloc: shape needs more scratch
+                                     than ATTN_NOALLOC_SCRATCH_BYTES            */
 
 /* Sticky device-side error bits, read by attn_check_error().  When a
  * sequence trips one, none of its output rows are written. */
@@ -187,6 +189,42 @@ void attn_destroy(attn_plan_t plan);
 
 /* Static message for an ATTN_* return code. */
 const char *attn_strerror(int code);
+
+/*
+ * attn_run_noalloc -- one attention call for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is a convenience of
+ * this library.
+ *
+ * Who needs it: a caller whose host framework owns the device memory budget
+ * through its own pool allocator (a raw cudaMalloc by a library escapes the
+ * pool's accounting and can fail once the pool holds the device), or a caller
+ * on a latency-critical path where cudaMalloc / cudaFree may synchronise the
+ * device.  Such callers cannot make a plan, since attn_plan allocates.
+ *
+ * Arguments: the shape (B_max, s_max, Hq, Hkv, D, max_q; same meaning and
+ * limits as attn_plan) followed by the tensors and stream of attn_run (same
+ * layout, alignment and ownership rules).  Results match attn_run within the
+ * library's tolerance; the CUDA-core split kernel is used for every shape.
+ *
+ * Scratch: a file-scope device array of ATTN_NOALLOC_SCRATCH_BYTES inside the
+ * library, held by every GPU that loads the library until the process exits.
+ * A shape whose split partials would not fit is rejected with
+ * ATTN_E_SCRATCH_LIMIT and nothing is launched.  The call allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library routine).
+ *
+ * The first call on each device looks up the array's device address and sets
+ * a kernel attribute; make that first call before any stream capture begins.
+ * All calls on a device share the array and leave their contents in it; each
+ * call clears the parts that must start at zero on its own stream.  Calls
+ * that overlap on the GPU race on the array: order them (one stream, or
+ * events).  Device-detected length errors leave those rows unwritten, as in
+ * attn_run, but are not reported (there is no plan to read them from).
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (4u << 20)
+int attn_run_noalloc(int B_max, int s_max, int Hq, int Hkv, int D, int max_q,
+                     const void *q, const void *k, const void *v,
+                     const int32_t *cu_q, const int32_t *cu_k, void *out,
+                     float *lse, void *stream);
 
 #ifdef __cplusplus
 }

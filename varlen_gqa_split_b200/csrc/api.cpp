@@ -93,6 +93,7 @@ ATTN_EXPORT const char *attn_strerror(int code) {
     case ATTN_E_NOMEM: return "device allocation failed";
     case ATTN_E_DEVICE: return "current device differs from the plan's device";
     case ATTN_E_NO_DEVICE: return "no usable sm_100 device";
+    case ATTN_E_SCRATCH_LIMIT: return "shape needs more scratch than the fixed no-allocation array holds";
     default: return "unknown error code";
     }
 }
