@@ -89,6 +89,10 @@ typedef struct {
     int variant;   /* ATTN_VARIANT_*                                            */
     int stages;    /* pipeline depth of the tensor-core path: 2..8              */
     int combine;   /* ATTN_COMBINE_*                                            */
+    int ctas;      /* tensor-core path: blocks sharing the tile space; >= 1     */
+    int deterministic; /* 1: bitwise-repeatable results (static tile shares);
+                          0: blocks that share a unit balance it between them
+                          at run time, results equal within rounding           */
 } attn_overrides;
 
 /* What the planner chose (attn_plan_info). */
@@ -96,13 +100,18 @@ typedef struct {
     int B_max, s_max, Hq, Hkv, D, max_q;
     int G;                 /* Hq / Hkv                                          */
     int variant;           /* ATTN_VARIANT_SIMT or ATTN_VARIANT_MMA             */
-    int nsplit;            /* KV chunks per (sequence, KV head)                  */
-    int chunk;             /* keys per chunk (multiple of block_n)               */
+    int nsplit;            /* SIMT path: KV chunks per (sequence, KV head); 0 on
+                              the tensor-core path, whose split points follow
+                              the balanced per-block shares                      */
+    int chunk;             /* SIMT path: keys per chunk (multiple of block_n)    */
     int block_n;           /* keys per tile                                      */
     int stages;            /* pipeline stages (tensor-core path)                 */
     int rows_per_block;    /* query rows (G * q tokens) one block handles        */
     int row_tiles;         /* blocks along the row axis per KV head              */
-    int grid_x, grid_y, grid_z;   /* split-kernel grid: (nsplit, Hkv*row_tiles, B_max) */
+    int grid_x, grid_y, grid_z;   /* split-kernel grid: SIMT (nsplit, Hkv*row_tiles,
+                              B_max); tensor-core (ctas, 1, 1)                    */
+    int ctas;              /* tensor-core path: persistent blocks (0 on SIMT)    */
+    int deterministic;     /* 1 if results are bitwise repeatable for this plan  */
     int combine;           /* ATTN_COMBINE_KERNEL or ATTN_COMBINE_FUSED          */
     int combine_blocks;    /* combine-kernel blocks (0 unless a combine kernel runs) */
     int smem_bytes;        /* dynamic shared memory of the split kernel          */

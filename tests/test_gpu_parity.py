@@ -102,17 +102,37 @@ def test_continuous_batching_one_graph_many_steps():
 # ------------------------------------------------------------ split-count invariance
 
 @pytest.mark.parametrize("combine", [vg.ATTN_COMBINE_FUSED, vg.ATTN_COMBINE_KERNEL])
-@pytest.mark.parametrize("variant", [SIMT, MMA])
-def test_nsplit_invariance(variant, combine):
+def test_nsplit_invariance_simt(combine):
     sh = W.Shape("mid", B=4, Hq=64, Hkv=8, D=128, max_q=1, s_max=4096)
     batch = W.make_batch(sh, [1, 1, 1, 1], [4096, 1000, 77, 0], seed=3, gen_device="cuda")
     ref_o, ref_l = oracle_full(batch)
     cov = covered_rows(batch)
     outs = []
     for ns in (1, 2, 3, 8, 32, 64):
-        plan = plan_for(sh, variant=variant, nsplit=ns, combine=combine)
+        plan = plan_for(sh, variant=SIMT, nsplit=ns, combine=combine)
         assert plan.info["nsplit"] == ns
         assert plan.info["combine"] == (0 if ns == 1 else combine)
+        out, lse = run_gpu(plan, batch)
+        compare_full(out, lse, ref_o, ref_l, cov)
+        outs.append(out.float().numpy())
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= 2 * ATOL_OUT
+
+
+@pytest.mark.parametrize("stages,det", [(0, 0), (0, 1), (2, 0), (3, 1)])
+def test_block_count_invariance_mma(stages, det):
+    """The persistent tensor-core path at 1 .. 2 x SM-count blocks: from one
+    block that finishes every unit itself to shares that cut every unit many
+    times (several partials per unit, merged by the last block to finish)."""
+    sh = W.Shape("mid", B=4, Hq=64, Hkv=8, D=128, max_q=1, s_max=4096)
+    batch = W.make_batch(sh, [1, 1, 1, 1], [4096, 1000, 77, 0], seed=3, gen_device="cuda")
+    ref_o, ref_l = oracle_full(batch)
+    cov = covered_rows(batch)
+    outs = []
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for ctas in (1, 2, 3, 7, 37, sms, 2 * sms):
+        plan = plan_for(sh, variant=MMA, ctas=ctas, stages=stages, deterministic=det)
+        assert plan.info["ctas"] == ctas and plan.info["nsplit"] == 0
         out, lse = run_gpu(plan, batch)
         compare_full(out, lse, ref_o, ref_l, cov)
         outs.append(out.float().numpy())
@@ -133,16 +153,34 @@ def test_variants_agree():
     assert np.abs(l1[fin] - l2[fin]).max() <= 2 * ATOL_LSE
 
 
-@pytest.mark.parametrize("combine", [vg.ATTN_COMBINE_FUSED, vg.ATTN_COMBINE_KERNEL])
-def test_repeat_runs_bitwise_equal(combine):
-    # a fixed plan is deterministic: the merge order does not depend on which
-    # block of a unit finishes last
+@pytest.mark.parametrize("kw", [{"deterministic": 1},
+                                {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_FUSED},
+                                {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_KERNEL}])
+def test_repeat_runs_bitwise_equal(kw):
+    # a deterministic plan repeats bit for bit: fixed tile shares and a fixed
+    # merge order, whichever block finishes last
     batch = W.workload("long", gen_device="cuda")
-    plan = plan_for(batch.shape, combine=combine)
+    plan = plan_for(batch.shape, **kw)
+    assert plan.info["deterministic"] == 1
     runs = [run_gpu(plan, batch) for _ in range(3)]
     for o, l in runs[1:]:
         assert torch.equal(o.view(torch.int16), runs[0][0].view(torch.int16))
         assert torch.equal(l.view(torch.int32), runs[0][1].view(torch.int32))
+
+
+def test_dynamic_balance_repeats_within_rounding():
+    # with run-time balancing inside cut units, repeated calls agree with each
+    # other and with the oracle within the tolerance, not bit for bit
+    batch = W.workload("long", gen_device="cuda")
+    plan = plan_for(batch.shape)
+    assert plan.info["deterministic"] == 0
+    ref_o, ref_l = oracle_full(batch)
+    cov = covered_rows(batch)
+    runs = [run_gpu(plan, batch) for _ in range(4)]
+    for o, l in runs:
+        compare_full(o, l, ref_o, ref_l, cov)
+    for o, _ in runs[1:]:
+        assert (o.float() - runs[0][0].float()).abs().max().item() <= 2 * ATOL_OUT
 
 
 # ------------------------------------------------------------ placement and edge cases
@@ -172,20 +210,25 @@ def test_exhaustive_small_lengths_placement(variant):
     compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
 
 
-@pytest.mark.parametrize("combine", [vg.ATTN_COMBINE_FUSED, vg.ATTN_COMBINE_KERNEL])
-@pytest.mark.parametrize("variant,nsplit", [(SIMT, 1), (SIMT, 3), (MMA, 1), (MMA, 2), (MMA, 5)])
-def test_ragged_multi_tile_placement(variant, nsplit, combine):
-    """Lengths spanning several 64-key tiles and chunks, short sequences whose
-    tile starts before the buffer (negative TMA coordinates), Lq up to 2."""
-    rng = np.random.default_rng(5 + nsplit)
+@pytest.mark.parametrize("kw", [{"variant": SIMT, "nsplit": 1}, {"variant": SIMT, "nsplit": 3},
+                                {"variant": SIMT, "nsplit": 3, "combine": vg.ATTN_COMBINE_KERNEL},
+                                {"variant": MMA, "ctas": 1}, {"variant": MMA, "ctas": 5},
+                                {"variant": MMA, "ctas": 64}, {"variant": MMA},
+                                {"variant": MMA, "ctas": 64, "deterministic": 1}])
+def test_ragged_multi_tile_placement(kw):
+    """Lengths spanning several 64-key tiles, units cut across blocks, short
+    sequences whose tile starts before the buffer (negative TMA
+    coordinates), sequences without keys or queries, Lq up to 2."""
+    rng = np.random.default_rng(5 + len(kw))
     B = 40
     lq = rng.integers(0, 3, B)
     lk = rng.integers(0, 330, B)
     lk[:3] = [1, 63, 64]
     lk[3:6] = [65, 0, 129]
+    lq[6] = 0
     sh = W.Shape("ragged_mt", B=B + 2, Hq=16, Hkv=2, D=128, max_q=2, s_max=330)
     batch = W.make_batch(sh, lq, lk, seed=7, gen_device="cuda")
-    plan = plan_for(sh, variant=variant, nsplit=nsplit, combine=combine)
+    plan = plan_for(sh, **kw)
     out, lse = run_gpu(plan, batch, extra_q_rows=1)
     ref_o, ref_l = oracle_full(batch)
     compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
@@ -207,7 +250,7 @@ def test_large_magnitude_scores(variant):
     sh = W.Shape("big", B=2, Hq=8, Hkv=1, D=128, max_q=1, s_max=2048)
     batch = W.make_batch(sh, [1, 1], [2048, 513], seed=4, gen_device="cuda")
     batch.q = (batch.q.float() * 30).to(torch.bfloat16)
-    plan = plan_for(sh, variant=variant, nsplit=4)
+    plan = plan_for(sh, variant=variant, **({"nsplit": 4} if variant == SIMT else {"ctas": 9}))
     out, lse = run_gpu(plan, batch)
     ref_o, ref_l = oracle_full(batch)
     compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
@@ -216,11 +259,10 @@ def test_large_magnitude_scores(variant):
 def test_plan_choices_follow_the_split_rule():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     long_plan = plan_for(W.SHAPES["long"])
-    assert long_plan.info["nsplit"] > 1 and long_plan.info["variant"] == MMA
-    assert long_plan.info["grid_x"] * long_plan.info["grid_y"] >= sms
-    ragged_plan = plan_for(W.SHAPES["ragged"])
-    assert ragged_plan.info["nsplit"] == 1          # B * Hkv = 512 blocks already fill the SMs
-    assert ragged_plan.info["scratch_bytes"] <= 1024
+    assert long_plan.info["variant"] == MMA and long_plan.info["ctas"] == sms
+    ragged_simt = plan_for(W.SHAPES["ragged"], variant=SIMT)
+    assert ragged_simt.info["nsplit"] == 1          # B * Hkv = 512 blocks already fill the SMs
+    assert ragged_simt.info["scratch_bytes"] <= 1024
     sq = plan_for(W.SHAPES["shortq"])
     assert sq.info["variant"] == SIMT
 
@@ -277,6 +319,8 @@ def test_host_side_errors_launch_nothing():
         vg.Plan(1, 64, 4, 1, 96, 1)                         # unsupported head dim
     with pytest.raises(vg.AttnError):
         vg.Plan(1, 64, 64, 8, 128, 4, variant=MMA)         # 32 rows > tensor-core path limit
+    with pytest.raises(vg.AttnError):
+        vg.Plan(1, 64, 8, 1, 128, 1, variant=MMA, nsplit=2)  # split count belongs to the SIMT grid
     handle = plan.handle
     plan.close()
     assert L.attn_run(handle, q.data_ptr(), k.data_ptr(), k.data_ptr(), cu.data_ptr(), cu.data_ptr(),

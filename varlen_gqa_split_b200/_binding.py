@@ -31,13 +31,15 @@ EXPORTED = ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_che
 
 class Overrides(ctypes.Structure):
     _fields_ = [("nsplit", ctypes.c_int), ("block_n", ctypes.c_int), ("variant", ctypes.c_int),
-                ("stages", ctypes.c_int), ("combine", ctypes.c_int)]
+                ("stages", ctypes.c_int), ("combine", ctypes.c_int), ("ctas", ctypes.c_int),
+                ("deterministic", ctypes.c_int)]
 
 
 class PlanDesc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "B_max", "s_max", "Hq", "Hkv", "D", "max_q", "G", "variant", "nsplit", "chunk", "block_n",
-        "stages", "rows_per_block", "row_tiles", "grid_x", "grid_y", "grid_z", "combine", "combine_blocks",
+        "stages", "rows_per_block", "row_tiles", "grid_x", "grid_y", "grid_z", "ctas", "deterministic", "combine",
+        "combine_blocks",
         "smem_bytes", "num_sms")] + [("scratch_bytes", ctypes.c_size_t)]
 
 
@@ -99,14 +101,16 @@ class Plan:
     """A plan: launch shape, split count and scratch fixed from constants.
 
     Plan(B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
-    stages=0, combine=0) -- the keyword choices override the planner (0 = its own)."""
+    stages=0, combine=0, ctas=0, deterministic=0) -- the keyword choices
+    override the planner (0 = its own)."""
 
     def __init__(self, B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
-                 stages=0, combine=0):
+                 stages=0, combine=0, ctas=0, deterministic=0):
         L = lib()
         h = ctypes.c_void_p()
-        if nsplit or block_n or variant or stages or combine:
-            o = Overrides(int(nsplit), int(block_n), int(variant), int(stages), int(combine))
+        if nsplit or block_n or variant or stages or combine or ctas or deterministic:
+            o = Overrides(int(nsplit), int(block_n), int(variant), int(stages), int(combine), int(ctas),
+                          int(deterministic))
             rc = L.attn_plan_ex(ctypes.byref(h), int(B_max), int(s_max), int(Hq), int(Hkv), int(D),
                                 int(max_q), ctypes.byref(o))
         else:

@@ -33,6 +33,7 @@ struct attn_plan_s {
     uint32_t *err;
     uint32_t *ticket;          // fused-merge arrival counters
     size_t ticket_bytes;
+    int merge_bytes;           // tensor-core path: shared bytes of the merge area
     float *o_part;
     float2 *ml_part;
 };
@@ -110,9 +111,11 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_E_NO_DEVICE;
-    int major = 0, sms = 0;
+    int major = 0, sms = 0, smem_sm = 0, smem_block = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_block, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return ATTN_E_NO_DEVICE;
     if (major != 10) return ATTN_E_NO_DEVICE;
 
@@ -130,81 +133,98 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     if (variant != ATTN_VARIANT_MMA && variant != ATTN_VARIANT_SIMT) return ATTN_E_INVALID_ARG;
     if (variant == ATTN_VARIANT_MMA && rows > 16) return ATTN_E_UNSUPPORTED;
     if (o && o->block_n && o->block_n != 64) return ATTN_E_UNSUPPORTED;
+    if (o && (o->nsplit < 0 || o->stages < 0 || o->ctas < 0)) return ATTN_E_INVALID_ARG;
+    if (o && o->combine && o->combine != ATTN_COMBINE_KERNEL && o->combine != ATTN_COMBINE_FUSED)
+        return ATTN_E_INVALID_ARG;
     d.variant = variant;
+    const int tiles_max = (s_max + 63) / 64;
 
     int NT = 1;
-    int per_sm = 1;
+    size_t n_ticket = 0, n_part = 0, part_rows = 0;
+    int merge_bytes = 0;
     if (variant == ATTN_VARIANT_MMA) {
+        // persistent: about one block per SM, each with a deep load ring; the
+        // split points follow the balanced per-block shares (nsplit and chunk
+        // do not apply) and the slot-parallel combine kernel merges cut units
+        if (o && (o->nsplit || o->combine == ATTN_COMBINE_FUSED)) return ATTN_E_UNSUPPORTED;
         NT = rows <= 8 ? 1 : 2;
         d.block_n = mma_block_n();
-        d.stages = o && o->stages ? o->stages : (D == 128 ? 3 : 4);
-        if (d.stages < 2 || d.stages > 8) return ATTN_E_INVALID_ARG;
+        const long long max_tiles = (long long)B_max * Hkv * tiles_max;
+        long long ctas = o && o->ctas ? o->ctas : sms;
+        ctas = std::min<long long>(ctas, std::max(1LL, max_tiles));
+        ctas = std::min<long long>(ctas, 65535);
+        d.ctas = (int)ctas;
+        const size_t fixed = mma_smem_bytes(D, NT, 0, d.ctas);
+        int stages = o && o->stages ? o->stages : (int)((smem_block - fixed) / mma_stage_bytes(D));
+        stages = std::min(stages, 8);
+        if (stages < 2 || mma_smem_bytes(D, NT, stages, d.ctas) > (size_t)smem_block) return ATTN_E_INVALID_ARG;
+        d.stages = stages;
         d.rows_per_block = 8 * NT;
         d.row_tiles = 1;
-        d.smem_bytes = (int)mma_smem_bytes(D, NT, d.stages);
-        if (mma_prepare(D, NT, d.stages) != cudaSuccess) return ATTN_E_CUDA;
+        d.smem_bytes = (int)mma_smem_bytes(D, NT, stages, d.ctas);
+        merge_bytes = (int)mma_merge_bytes(D, NT, d.ctas);
+        d.nsplit = 0;
+        d.chunk = 0;
+        d.grid_x = d.ctas;
+        d.grid_y = 1;
+        d.grid_z = 1;
+        d.deterministic = o && o->deterministic ? 1 : 0;
+        d.combine = ATTN_COMBINE_KERNEL;     // slot-parallel combine, programmatic dependent launch
+        d.combine_blocks = 2 * d.ctas;
+        n_ticket = 2 * (size_t)B_max * Hkv;  // tile-claim counters of cut units (64-bit each)
+        n_part = 2 * (size_t)d.ctas;       // two partial slots per block
+        part_rows = d.rows_per_block;
+        if (mma_prepare(D, NT, stages, d.ctas) != cudaSuccess) return ATTN_E_CUDA;
     } else {
+        if (o && o->ctas) return ATTN_E_UNSUPPORTED;
+        d.deterministic = 1;                 // fixed grid, fixed merge order
         d.block_n = kSimtBlockN;
         d.stages = 2;
         d.rows_per_block = kSimtRowsPerBlock;
         d.row_tiles = (int)((rows + kSimtRowsPerBlock - 1) / kSimtRowsPerBlock);
         d.smem_bytes = (int)simt_smem_bytes(D);
+        if ((long long)Hkv * d.row_tiles > 65535) return ATTN_E_INVALID_ARG;
         if (simt_prepare(D) != cudaSuccess) return ATTN_E_CUDA;
-    }
-    if ((long long)Hkv * d.row_tiles > 65535) return ATTN_E_INVALID_ARG;
-    {
         // resident blocks per SM, from shared memory (the binding limit here)
-        int smem_sm = 0;
-        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-        per_sm = std::max(1, smem_sm / (d.smem_bytes + 1024));
-        per_sm = std::min(per_sm, 4);
+        const int per_sm = std::min(4, std::max(1, smem_sm / (d.smem_bytes + 1024)));
+        // Split count: fill the device (about per_sm blocks per SM), capped by
+        // the tile count; fall back to one direct-write pass when the
+        // (sequence, KV head, row tile) units alone already fill it (AstrAI
+        // commit log, split-KV commit).
+        const long long units = (long long)B_max * Hkv * d.row_tiles;
+        const long long target = (long long)sms * per_sm;
+        long long ns;
+        if (o && o->nsplit)
+            ns = o->nsplit;
+        else if (units >= target)
+            ns = 1;
+        else
+            ns = (target + units - 1) / units;
+        ns = std::max(1LL, std::min<long long>(ns, std::min(tiles_max, 1024)));
+        const int tiles_per_chunk = (int)((tiles_max + ns - 1) / ns);
+        d.chunk = tiles_per_chunk * d.block_n;
+        d.nsplit = (s_max + d.chunk - 1) / d.chunk;
+        d.grid_x = d.nsplit;
+        d.grid_y = Hkv * d.row_tiles;
+        d.grid_z = B_max;
+        // partials merged by the last block of each unit (one launch per call)
+        // when its shared memory holds the merge tables, else by a second kernel
+        if (d.nsplit > 1) {
+            const size_t need = (size_t)d.rows_per_block * (d.nsplit + 1) * 8;
+            const int want = o && o->combine ? o->combine : ATTN_COMBINE_FUSED;
+            d.combine = (want == ATTN_COMBINE_FUSED && need <= simt_merge_capacity(D)) ? ATTN_COMBINE_FUSED
+                                                                                      : ATTN_COMBINE_KERNEL;
+            n_part = (size_t)B_max * max_q * Hq * d.nsplit;
+            part_rows = 1;
+            if (d.combine == ATTN_COMBINE_FUSED) n_ticket = (size_t)B_max * Hkv * d.row_tiles;
+        }
     }
 
-    // Split count: fill the device (about per_sm blocks per SM), capped by the
-    // tile count; fall back to one direct-write pass when the (sequence, KV
-    // head, row tile) units alone already fill it (AstrAI commit log,
-    // split-KV commit).
-    const long long units = (long long)B_max * Hkv * d.row_tiles;
-    const long long target = (long long)sms * per_sm;
-    const int tiles_max = (s_max + d.block_n - 1) / d.block_n;
-    long long ns;
-    if (o && o->nsplit) {
-        if (o->nsplit < 1) return ATTN_E_INVALID_ARG;
-        ns = o->nsplit;
-    } else if (units >= target) {
-        ns = 1;
-    } else {
-        ns = (target + units - 1) / units;
-    }
-    ns = std::max(1LL, std::min<long long>(ns, std::min(tiles_max, 1024)));
-    const int tiles_per_chunk = (int)((tiles_max + ns - 1) / ns);
-    d.chunk = tiles_per_chunk * d.block_n;
-    d.nsplit = (s_max + d.chunk - 1) / d.chunk;
-    d.grid_x = d.nsplit;
-    d.grid_y = Hkv * d.row_tiles;
-    d.grid_z = B_max;
-
-    // how split partials are merged: by the last block of each unit (one
-    // launch per call) when its shared memory holds the merge tables, else by
-    // a second kernel
-    int combine = 0;
-    if (d.nsplit > 1) {
-        const size_t need = (size_t)d.rows_per_block * (d.nsplit + 1) * 8;
-        const size_t cap = variant == ATTN_VARIANT_MMA ? mma_merge_capacity(D, d.stages) : simt_merge_capacity(D);
-        const int want = o && o->combine ? o->combine : ATTN_COMBINE_FUSED;
-        if (want != ATTN_COMBINE_KERNEL && want != ATTN_COMBINE_FUSED) return ATTN_E_INVALID_ARG;
-        combine = (want == ATTN_COMBINE_FUSED && need <= cap) ? ATTN_COMBINE_FUSED : ATTN_COMBINE_KERNEL;
-    }
-    d.combine = combine;
-
-    // scratch: error word, merge tickets, then (nsplit > 1) O partials and
-    // (m, l) partials
-    const size_t n_part = d.nsplit > 1 ? (size_t)B_max * max_q * Hq * d.nsplit : 0;
-    const size_t n_ticket = combine == ATTN_COMBINE_FUSED ? (size_t)B_max * Hkv * d.row_tiles : 0;
+    // scratch: error word, merge tickets, O partials, (m, l) partials
     const size_t off_t = 256;
     const size_t off_o = align_up(off_t + n_ticket * sizeof(uint32_t), 256);
-    const size_t off_ml = align_up(off_o + n_part * D * sizeof(float), 256);
-    const size_t total = align_up(off_ml + n_part * sizeof(float2), 256);
+    const size_t off_ml = align_up(off_o + n_part * part_rows * D * sizeof(float), 256);
+    const size_t total = align_up(off_ml + n_part * part_rows * sizeof(float2), 256);
     d.scratch_bytes = total;
 
     attn_plan_s *p = new (std::nothrow) attn_plan_s{};
@@ -212,6 +232,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     p->d = d;
     p->device = dev;
     p->NT = NT;
+    p->merge_bytes = merge_bytes;
     p->scale_log2 = (float)((1.0 / std::sqrt((double)D)) * 1.4426950408889634);
     if (cudaMalloc(&p->scratch, total) != cudaSuccess) {
         cudaGetLastError();
@@ -228,7 +249,6 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         delete p;
         return ATTN_E_CUDA;
     }
-    d.combine_blocks = 0;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         g_plans.insert(p);
@@ -240,7 +260,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
             return rc;
         }
     }
-    if (combine == ATTN_COMBINE_KERNEL) {
+    if (d.combine == ATTN_COMBINE_KERNEL && variant == ATTN_VARIANT_SIMT) {
         Params tmp{};
         tmp.B_max = B_max;
         tmp.max_q = max_q;
@@ -249,10 +269,10 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     }
     if (std::getenv("VGQA_LOG"))
         std::fprintf(stderr,
-                     "[vgqa] plan B_max=%d s_max=%d Hq=%d Hkv=%d D=%d max_q=%d: variant=%d nsplit=%d "
-                     "chunk=%d grid=(%d,%d,%d) smem=%d stages=%d per_sm=%d combine=%d scratch=%zu\n",
-                     B_max, s_max, Hq, Hkv, D, max_q, p->d.variant, p->d.nsplit, p->d.chunk, p->d.grid_x,
-                     p->d.grid_y, p->d.grid_z, p->d.smem_bytes, p->d.stages, per_sm, p->d.combine,
+                     "[vgqa] plan B_max=%d s_max=%d Hq=%d Hkv=%d D=%d max_q=%d: variant=%d nsplit=%d chunk=%d "
+                     "ctas=%d grid=(%d,%d,%d) smem=%d stages=%d combine=%d scratch=%zu\n",
+                     B_max, s_max, Hq, Hkv, D, max_q, p->d.variant, p->d.nsplit, p->d.chunk, p->d.ctas,
+                     p->d.grid_x, p->d.grid_y, p->d.grid_z, p->d.smem_bytes, p->d.stages, p->d.combine,
                      p->d.scratch_bytes);
     *out = p;
     return ATTN_OK;
@@ -305,7 +325,11 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
     p.row_tiles = d.row_tiles;
     p.scale_log2 = plan->scale_log2;
     p.ticket = plan->ticket;
+    p.claim = reinterpret_cast<unsigned long long *>(plan->ticket);
     p.fused = d.combine == ATTN_COMBINE_FUSED;
+    p.merge_bytes = plan->merge_bytes;
+    p.ctas_max = d.ctas;
+    p.dynamic = d.variant == ATTN_VARIANT_MMA && !d.deterministic;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(d.grid_x, d.grid_y, d.grid_z);
@@ -315,12 +339,12 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
         if (encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n) != ATTN_OK ||
             encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n) != ATTN_OK)
             return ATTN_E_CUDA;
-        e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, grid, s);
+        e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, d.ctas, s);
     } else {
         e = launch_split_simt(p, grid, s);
     }
     if (e != cudaSuccess) return ATTN_E_CUDA;
-    if (d.combine == ATTN_COMBINE_KERNEL) {
+    if (d.combine == ATTN_COMBINE_KERNEL && d.variant == ATTN_VARIANT_SIMT) {
         e = launch_combine(p, s);
         if (e != cudaSuccess) return ATTN_E_CUDA;
     }

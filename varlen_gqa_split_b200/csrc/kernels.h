@@ -17,14 +17,16 @@ cudaError_t launch_split_simt(const Params &p, dim3 grid, cudaStream_t stream);
 constexpr int kSimtRowsPerBlock = 16;
 constexpr int kSimtBlockN = 64;
 
-// TMA-fed tensor-core split kernel, NT = ceil(G * max_q / 8) in {1, 2}
-size_t mma_smem_bytes(int D, int NT, int stages);
-size_t mma_merge_capacity(int D, int stages);
+// Persistent TMA-fed tensor-core split kernel, NT = ceil(G * max_q / 8) in
+// {1, 2}, `ctas` blocks sharing the flattened tile space
+size_t mma_stage_bytes(int D);
+size_t mma_merge_bytes(int D, int NT, int ctas);
+size_t mma_smem_bytes(int D, int NT, int stages, int ctas);
 int mma_block_n();
 int mma_threads();
-cudaError_t mma_prepare(int D, int NT, int stages);
+cudaError_t mma_prepare(int D, int NT, int stages, int ctas);
 cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUtensorMap &tm_v, int NT,
-                             int stages, dim3 grid, cudaStream_t stream);
+                             int stages, int ctas, cudaStream_t stream);
 
 // log-sum-exp merge of the split partials
 int combine_blocks(const Params &p);

@@ -20,6 +20,7 @@ struct Params {
     float2 *ml_part;           // [B_max, max_q, Hq, nsplit]     (m, l) base-2
     uint32_t *err;             // sticky ATTN_DEV_ERR_* bits
     uint32_t *ticket;          // [B_max * Hkv * row_tiles] arrival counters (fused merge)
+    unsigned long long *claim; // [B_max * Hkv] tile claims of cut units (tensor-core path)
     int B_max, s_max, Hq, Hkv, D, max_q, G;
     int nsplit;                // chunks per (sequence, KV head)
     int chunk;                 // keys per chunk
@@ -27,6 +28,9 @@ struct Params {
     int row_tiles;             // row blocks per KV head
     float scale_log2;          // (1/sqrt(D)) * log2(e)
     int fused;                 // nsplit > 1: the last block of a unit merges it
+    int merge_bytes;           // tensor-core path: shared bytes of the merge area
+    int ctas_max;              // tensor-core path: blocks of the launch (merge table size)
+    int dynamic;               // tensor-core path: blocks sharing a cut unit claim its tiles
 };
 
 }  // namespace vgqa
