@@ -171,7 +171,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         d.deterministic = o && o->deterministic ? 1 : 0;
         d.combine = ATTN_COMBINE_KERNEL;     // slot-parallel combine, programmatic dependent launch
         d.combine_blocks = 2 * d.ctas;
-        n_ticket = 2 * (size_t)B_max * Hkv;  // tile-claim counters of cut units (64-bit each)
+        n_ticket = 3 * (size_t)B_max * Hkv;  // per cut unit: tile claims (64-bit), part count
         n_part = 2 * (size_t)d.ctas;       // two partial slots per block
         part_rows = d.rows_per_block;
         if (mma_prepare(D, NT, stages, d.ctas) != cudaSuccess) return ATTN_E_CUDA;
@@ -326,6 +326,7 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
     p.scale_log2 = plan->scale_log2;
     p.ticket = plan->ticket;
     p.claim = reinterpret_cast<unsigned long long *>(plan->ticket);
+    p.done = plan->ticket + 2 * (size_t)d.B_max * d.Hkv;
     p.fused = d.combine == ATTN_COMBINE_FUSED;
     p.merge_bytes = plan->merge_bytes;
     p.ctas_max = d.ctas;

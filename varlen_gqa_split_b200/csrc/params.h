@@ -21,6 +21,7 @@ struct Params {
     uint32_t *err;             // sticky ATTN_DEV_ERR_* bits
     uint32_t *ticket;          // [B_max * Hkv * row_tiles] arrival counters (fused merge)
     unsigned long long *claim; // [B_max * Hkv] tile claims of cut units (tensor-core path)
+    uint32_t *done;            // [B_max * Hkv] parts written / merges started per cut unit
     int B_max, s_max, Hq, Hkv, D, max_q, G;
     int nsplit;                // chunks per (sequence, KV head)
     int chunk;                 // keys per chunk

@@ -46,11 +46,11 @@
 //
 // Combine kernel: one block per partial slot, launched as a programmatic
 // dependent of the split kernel.  It recomputes the schedule from cu_seqlens
-// while the split kernel runs, then waits for the split kernel's results
-// (griddepcontrol.wait) and merges one column slice of its cut unit: the n
-// blocks of a cut unit merge it together, each reading 1/n of the partial
-// data, so the merge is spread over as many SMs as wrote it (one SM can pull
-// only a few tens of GB/s from L2, too little to merge a unit alone).
+// while the split kernel runs, waits only for the parts of its own unit, and
+// merges one column slice of it: the n blocks of a cut unit merge it
+// together, each reading 1/n of the partial data, so the merge is spread over
+// as many SMs as wrote it (one SM can pull only a few tens of GB/s from L2,
+// too little to merge a unit alone).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -677,6 +677,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             }
         }
         named_sync(kBarConsumers, kConsumers);     // warp-merge buffers free for the next unit
+        // publish the part: the combine block merging this unit waits for all n
+        if (!whole && tid == 0) red_add_release_gpu(p.done + (long long)cur.b * p.Hkv + cur.hk, 1u);
 
         if (!has_nxt) break;
         cur = nxt;
@@ -693,18 +695,24 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
 }
 
 // Combine: block 2c + k merges slice (c - c_first) of the unit block c cut at
-// its start (k = 0) or end (k = 1), if any.  Everything before
-// griddepcontrol.wait depends only on cu_seqlens and runs while the split
-// kernel is still streaming.
+// its start (k = 0) or end (k = 1), if any.  The block is launched as a
+// programmatic dependent of the split kernel, so it computes the schedule
+// while the split kernel streams; it then waits (bounded) only for the n parts
+// of its own unit, whose writers each add 1 (release) to the unit's count, so
+// a unit is merged as soon as its last part lands rather than when the whole
+// split grid ends.  After merging, each of the unit's n combine blocks adds 1
+// again; the one that brings the count to 2n resets it for the next call.
 template <int D, int NT>
-__global__ void __launch_bounds__(128) combine_mma_kernel(const Params p, const int C) {
+__global__ void __launch_bounds__(128, 4) combine_mma_kernel(const Params p, const int C) {
     constexpr int ROWS = 8 * NT;
     constexpr int kCols = D / 4;
     constexpr int kT = 128;
+    constexpr int kBatch = 12;             // loads in flight per thread (register budget)
     extern __shared__ __align__(16) uint8_t csm[];
     __shared__ long long scan[8];
     __shared__ long long first[3];
-    const int tid = threadIdx.x;
+    __shared__ int ok_flag;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int c = blockIdx.x >> 1, k = blockIdx.x & 1;
 
     Share sh;
@@ -726,57 +734,98 @@ __global__ void __launch_bounds__(128) combine_mma_kernel(const Params p, const 
     const int G = p.G, R = G * seg.s.Lq;
     const int items = R * kCols;
     const int per = (items + n - 1) / n;
-    const int it_lo = (c - c_first) * per, it_hi = min(items, it_lo + per);
-    if (it_lo >= it_hi) return;
+    const int it_lo = min(items, (c - c_first) * per), it_hi = min(items, it_lo + per);
+    const long long u = (long long)seg.b * p.Hkv + seg.hk;
+
     int *slots = reinterpret_cast<int *>(csm);                         // [n]
     for (int j = tid; j < n; j += kT) slots[j] = slot_of(c_first + j, seg.Pu, T, Ce);
+
+    // wait for the unit's n parts (acquire pairs with the writers' release)
+    if (tid == 0) {
+        int ok = 1;
+        if (ld_acquire_gpu(p.done + u) < (uint32_t)n) {
+            const unsigned long long t0 = globaltimer();
+            while (ld_acquire_gpu(p.done + u) < (uint32_t)n) {
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(256);
+            }
+        }
+        ok_flag = ok;
+        if (ok && c == c_first) p.claim[u] = 0ull;                      // claims, next call
+    }
     __syncthreads();
+    if (!ok_flag) return;
 
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // the split kernel's partials are visible
-    if (c == c_first && tid == 0) p.claim[(long long)seg.b * p.Hkv + seg.hk] = 0ull;  // claims, next call
-
-    // one item (row, 4 columns) per thread: all its parts' loads are issued
-    // before any is used (one L2 round trip per kBatch parts), then merged
-    // with a running max
-    constexpr int kBatch = 24;
-    for (int it = it_lo + tid; it < it_hi; it += kT) {
+    // two threads per item (row, 4 columns), each merging every other part
+    // with a running max, kBatch loads in flight; the pair then combines
+    const int n_work = 2 * (it_hi - it_lo);
+    for (int base = 0; base < n_work; base += kT) {
+        const int w = base + tid;
+        const bool valid = w < n_work;
+        const int it = it_lo + (valid ? w >> 1 : 0), half = w & 1;
         const int r = it / kCols, d4 = (it % kCols) * 4;
         float M = -INFINITY, L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j0 = 0; j0 < n; j0 += kBatch) {
-            float2 ml[kBatch];
-            float4 o[kBatch];
+        if (valid) {
+            for (int j0 = half; j0 < n; j0 += 2 * kBatch) {
+                float2 ml[kBatch];
+                float4 o[kBatch];
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                if (j0 + u < n) {
-                    const long long sl = slots[j0 + u];
-                    ml[u] = __ldcg(p.ml_part + sl * ROWS + r);
-                    o[u] = __ldcg(reinterpret_cast<const float4 *>(p.o_part + (sl * ROWS + r) * D + d4));
+                for (int q = 0; q < kBatch; ++q) {
+                    const int j = j0 + 2 * q;
+                    if (j < n) {
+                        const long long sl = slots[j];
+                        ml[q] = __ldcg(p.ml_part + sl * ROWS + r);
+                        o[q] = __ldcg(reinterpret_cast<const float4 *>(p.o_part + (sl * ROWS + r) * D + d4));
+                    }
                 }
-            }
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                if (j0 + u < n && ml[u].y > 0.f) {
-                    const float Mn = fmaxf(M, ml[u].x);
-                    const float a = ex2(M - Mn), w = ex2(ml[u].x - Mn);   // ex2(-inf) = 0
-                    acc.x = fmaf(acc.x, a, w * o[u].x);
-                    acc.y = fmaf(acc.y, a, w * o[u].y);
-                    acc.z = fmaf(acc.z, a, w * o[u].z);
-                    acc.w = fmaf(acc.w, a, w * o[u].w);
-                    L = fmaf(L, a, w * ml[u].y);
-                    M = Mn;
+                for (int q = 0; q < kBatch; ++q) {
+                    if (j0 + 2 * q < n && ml[q].y > 0.f) {
+                        const float Mn = fmaxf(M, ml[q].x);
+                        const float a = ex2(M - Mn), wq = ex2(ml[q].x - Mn);   // ex2(-inf) = 0
+                        acc.x = fmaf(acc.x, a, wq * o[q].x);
+                        acc.y = fmaf(acc.y, a, wq * o[q].y);
+                        acc.z = fmaf(acc.z, a, wq * o[q].z);
+                        acc.w = fmaf(acc.w, a, wq * o[q].w);
+                        L = fmaf(L, a, wq * ml[q].y);
+                        M = Mn;
+                    }
                 }
             }
         }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const int qi = r / G, h = seg.hk * G + r % G;
-        const long long tok = seg.s.q0 + qi;
-        uint2 pk;
-        pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-        pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-        *reinterpret_cast<uint2 *>(p.out + (tok * p.Hq + h) * D + d4) = pk;
-        if (d4 == 0) p.lse[tok * p.Hq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        // combine the pair (adjacent lanes)
+        const float M2 = __shfl_xor_sync(0xffffffffu, M, 1);
+        const float L2 = __shfl_xor_sync(0xffffffffu, L, 1);
+        float4 a2;
+        a2.x = __shfl_xor_sync(0xffffffffu, acc.x, 1);
+        a2.y = __shfl_xor_sync(0xffffffffu, acc.y, 1);
+        a2.z = __shfl_xor_sync(0xffffffffu, acc.z, 1);
+        a2.w = __shfl_xor_sync(0xffffffffu, acc.w, 1);
+        if (valid && half == 0) {
+            const float Mt = fmaxf(M, M2);
+            const float Mref = Mt == -INFINITY ? 0.f : Mt;
+            const float s1 = ex2(M - Mref), s2 = ex2(M2 - Mref);
+            const float Lt = L * s1 + L2 * s2;
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+            const int qi = r / G, h = seg.hk * G + r % G;
+            const long long tok = seg.s.q0 + qi;
+            uint2 pk;
+            pk.x = pack_bf16x2((acc.x * s1 + a2.x * s2) * inv, (acc.y * s1 + a2.y * s2) * inv);
+            pk.y = pack_bf16x2((acc.z * s1 + a2.z * s2) * inv, (acc.w * s1 + a2.w * s2) * inv);
+            *reinterpret_cast<uint2 *>(p.out + (tok * p.Hq + h) * D + d4) = pk;
+            if (d4 == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
+        }
     }
+    (void)lane;
+    __syncthreads();
+    // every combine block of the unit has seen its n parts once the count
+    // reaches 2n: the last one resets it
+    if (tid == 0 && atomicAdd(p.done + u, 1u) == (uint32_t)(2 * n - 1)) p.done[u] = 0u;
 }
 
 size_t combine_mma_smem(int /*NT*/, int ctas) {
