@@ -339,61 +339,82 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
 
     stream = torch.cuda.Stream(dev)
     # Timing.  A call whose inputs exceed L2 is timed in a pipeline: R copies
-    # of the inputs (together several times L2) and one captured graph per
-    # copy, replayed back to back, K calls between one pair of events -- the
-    # steady state of a decode step whose layers each read their own cache.
-    # A smaller call is timed alone: L2 flushed before each call and events
-    # captured inside the graph around the call.  The isolated per-call
-    # latency (flush, then one call) is reported for every workload.
+    # of the inputs (together several times L2), one per layer of a model, and
+    # one CUDA graph holding R calls, one per copy -- the attention calls of a
+    # decode step over the layers' own caches.  K calls = K/R replays (plus a
+    # shorter graph for a remainder) between one pair of events.  A smaller
+    # call is timed alone: L2 flushed before each call, events captured inside
+    # the graph around the call.  The isolated per-call latency (flush, then
+    # one call) is reported for every workload.
     cu_steps_h, step_bytes = step_cu_k(args.workload, batch)
-    cu_steps = torch.from_numpy(cu_steps_h).to(dev)
     n_var = len(step_bytes)
     pipelined = min(step_bytes) >= L2_BYTES
     n_copies = max(2, min(8, -(-4 * L2_BYTES // min(step_bytes)))) if pipelined else 1
     copies = [(q, k, v, out, lse)]
     for _ in range(n_copies - 1):
         copies.append((q.clone(), k.clone(), v.clone(), torch.empty_like(out), torch.empty_like(lse)))
+    # one cu_seqlens_k row per copy; with several length draws, the rows of
+    # the next n_copies draws are written in place before each replay
+    cu_ext = np.concatenate([cu_steps_h, cu_steps_h[:n_copies]]) if n_var > 1 else cu_steps_h
+    cu_steps = torch.from_numpy(cu_ext).to(dev)
+    cu_rows = cu_steps[:1].repeat(n_copies, 1).contiguous()
     in0 = torch.cuda.Event(enable_timing=True, external=True)
     in1 = torch.cuda.Event(enable_timing=True, external=True)
-    graphs = []
+
+    def capture(n_calls, events=False):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="global"):
+            if events:
+                in0.record(stream)
+            for r in range(n_calls):
+                qq, kk, vv, oo, ll = copies[r]
+                plan.run(qq, kk, vv, cu_q, cu_rows[r], oo, ll)
+            if events:
+                in1.record(stream)
+        return g
+
     with torch.cuda.stream(stream):
-        plan.run(q, k, v, cu_q, cu_k, out, lse)
+        plan.run(q, k, v, cu_q, cu_rows[0], out, lse)
         stream.synchronize()
-        for i, (qq, kk, vv, oo, ll) in enumerate(copies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream, capture_error_mode="global"):
-                if i == 0:
-                    in0.record(stream)
-                plan.run(qq, kk, vv, cu_q, cu_k, oo, ll)
-                if i == 0:
-                    in1.record(stream)
-            graphs.append(g)
+        g_iso = capture(1, events=True)
+        g_all = capture(n_copies) if pipelined else None
+        rem = args.steps % n_copies
+        g_rem = capture(rem) if pipelined and rem else None
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     o0 = torch.cuda.Event(enable_timing=True)
     o1 = torch.cuda.Event(enable_timing=True)
 
     def isolated_step():
         flush.zero_()
-        graphs[0].replay()
+        g_iso.replay()
         stream.synchronize()
         return in0.elapsed_time(in1)
+
+    def set_draws(j):
+        if n_var > 1:
+            s0 = (j * n_copies) % n_var
+            cu_rows.copy_(cu_steps[s0:s0 + n_copies], non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             isolated_step()
         iso_ms = [isolated_step() for _ in range(min(args.steps, 200))]
-        for i in range(args.warmup * n_copies):
-            graphs[i % n_copies].replay()
+        if pipelined:
+            for j in range(args.warmup):
+                set_draws(j)
+                g_all.replay()
         stream.synchronize()
         barrier(pg)
         torch.cuda.synchronize(dev)
         with ClockSampler(local) as clocks:
             if pipelined:
                 o0.record(stream)
-                for i in range(args.steps):
-                    if n_var > 1:
-                        cu_k.copy_(cu_steps[i % n_var], non_blocking=True)
-                    graphs[i % n_copies].replay()
+                for j in range(args.steps // n_copies):
+                    set_draws(j)
+                    g_all.replay()
+                if g_rem is not None:
+                    set_draws(args.steps // n_copies)
+                    g_rem.replay()
                 o1.record(stream)
                 stream.synchronize()
                 total_local_ms = o0.elapsed_time(o1)
@@ -485,9 +506,10 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
                        "l2": (f"inputs larger than L2: {n_copies} copies of the inputs ({n_copies} x "
                               f"{bytes_['total'] / 1e6:.0f} MB) used in turn" if pipelined else
                               "flushed before every timed call (512 MB write, outside the timed events)"),
-                       "timing": ("CUDA events around K back-to-back CUDA-graph replays of one attn_run each "
-                                  "(rotating input copies)" +
-                                  ("; before each replay a device-to-device copy writes that step's "
+                       "timing": (f"CUDA events around K attn_run calls, captured {n_copies} per CUDA graph "
+                                  f"(one per input copy, like the layers of a decode step) and replayed back "
+                                  f"to back" +
+                                  ("; before each replay one device-to-device copy writes the next draws' "
                                    "cu_seqlens_k in place (timed)" if n_var > 1 else "") if pipelined else
                                   "CUDA events captured inside the graph around the attn_run call, one replay "
                                   "per step after an L2 flush, summed"),
@@ -504,7 +526,7 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
                                  "value_gbs": bytes_["total"] / (statistics.median(iso_ms) * 1e-3) / 1e9,
                                  "how": "L2 flushed, then one call; CUDA events inside the captured graph"},
         }
-    del graphs
+    del g_iso, g_all, g_rem
     plan.close()
     return res
 
