@@ -314,14 +314,6 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     const int warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
 
-    // ------------------------------------------------------------ schedule
-    // the combine kernel may launch now: it only waits for this grid's results
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    Share sh;
-    if (!block_share(p, c, gridDim.x, tid, kThreads, c == 0, scan, first, sh)) return;
-    const long long lo = sh.lo, hi = sh.hi;
-    const int b_first = sh.b_first;
-    const long long pb_first = sh.pb_first;
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
@@ -330,6 +322,25 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
         flags[0] = 0;
         fence_barrier_init();
     }
+    if (tid == kConsumers) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    // Launched as a programmatic dependent, the block may start while the
+    // previous kernel in the stream still runs; everything above touches only
+    // this block's shared memory.  Wait for that kernel (it may write the
+    // inputs, and a previous call's combine resets the counters used below)
+    // before reading any global memory.  Only then may this call's combine
+    // kernel launch: it relies on the counters being reset.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // ------------------------------------------------------------ schedule
+    Share sh;
+    if (!block_share(p, c, gridDim.x, tid, kThreads, c == 0, scan, first, sh)) return;
+    const long long lo = sh.lo, hi = sh.hi;
+    const int b_first = sh.b_first;
+    const long long pb_first = sh.pb_first;
     __syncthreads();
 
     // ------------------------------------------------------------ producer
@@ -346,8 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     // (an empty stage carries the flag when the block got no tile of it).
     if (warp == kConsumerWarps) {
         if (lane == 0) {
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
             const uint64_t pol = l2_evict_first();
             OrderedWalker wk;
             wk.init(p, b_first, pb_first, lo, hi);
@@ -714,6 +723,9 @@ __global__ void __launch_bounds__(128, 4) combine_mma_kernel(const Params p, con
     __shared__ int ok_flag;
     const int tid = threadIdx.x, lane = tid & 31;
     const int c = blockIdx.x >> 1, k = blockIdx.x & 1;
+    // the next call's split kernel may launch now; it waits for this grid to
+    // complete before it reads anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     Share sh;
     if (!block_share(p, c, C, tid, kT, false, scan, first, sh)) return;
@@ -882,36 +894,31 @@ cudaError_t mma_prepare(int D, int NT, int stages, int ctas) {
 
 cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUtensorMap &tm_v, int NT,
                              int stages, int ctas, cudaStream_t stream) {
-    const size_t smem = mma_smem_bytes(p.D, NT, stages, ctas);
-    const dim3 grid(ctas);
-    if (p.D == 64) {
-        if (NT == 1)
-            split_mma_kernel<64, 1><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, p, stages);
-        else
-            split_mma_kernel<64, 2><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, p, stages);
-    } else {
-        if (NT == 1)
-            split_mma_kernel<128, 1><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, p, stages);
-        else
-            split_mma_kernel<128, 2><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, p, stages);
-    }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // the combine kernel follows as a programmatic dependent: its blocks may
-    // start (and compute the schedule) before the split kernel has finished
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(2 * ctas);
-    cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = combine_mma_smem(NT, ctas);
-    cfg.stream = stream;
+    // Both kernels are launched as programmatic dependents of what precedes
+    // them in the stream: the split kernel's blocks may become resident and
+    // set up while the previous kernel finishes (they wait for it before
+    // reading global memory), and the combine kernel's blocks start (and
+    // compute the schedule) before the split kernel has finished.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = mma_smem_bytes(p.D, NT, stages, ctas);
+    cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void *fn = combine_pick(p.D, NT);
-    void *args[] = {const_cast<Params *>(&p), &ctas};
-    return cudaLaunchKernelExC(&cfg, fn, args);
+    int st = stages;
+    void *split_args[] = {const_cast<CUtensorMap *>(&tm_k), const_cast<CUtensorMap *>(&tm_v),
+                          const_cast<Params *>(&p), &st};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, pick(p.D, NT), split_args);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(2 * ctas);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = combine_mma_smem(NT, ctas);
+    void *combine_args[] = {const_cast<Params *>(&p), &ctas};
+    return cudaLaunchKernelExC(&cfg, combine_pick(p.D, NT), combine_args);
 }
 
 }  // namespace vgqa
