@@ -437,7 +437,7 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     # bound on the split kernel's own rate.  Its share of device time is in the
     # committed ncu launch list.
     peak, peak_src = measured_peak()
-    kernel = {1: "split_simt_kernel", 2: "split_mma_kernel"}[info["variant"]]
+    kernel = {1: "split_simt_kernel", 2: "split_mma_kernel", 3: "split_tc_kernel"}[info["variant"]]
     achieved = timed_bytes / (total_ms * 1e-3) / 1e9
     traffic, traffic_note = recorded_traffic(args.workload, kernel)
     roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -68,7 +68,9 @@ extern "C" {
 /* Kernel variants (attn_overrides.variant / attn_plan_desc.variant). */
 #define ATTN_VARIANT_AUTO 0
 #define ATTN_VARIANT_SIMT 1   /* CUDA-core path, any row count               */
-#define ATTN_VARIANT_MMA 2    /* TMA-fed tensor-core path, G*max_q <= 16      */
+#define ATTN_VARIANT_MMA 2    /* TMA-fed warp-MMA path, G*max_q <= 16         */
+#define ATTN_VARIANT_TC 3     /* TMA-fed tcgen05 path (tensor memory),
+                                 G*max_q <= 128                              */
 
 /* How split partials are merged (attn_overrides.combine / attn_plan_desc.combine). */
 #define ATTN_COMBINE_AUTO 0
@@ -99,7 +101,7 @@ typedef struct {
 typedef struct {
     int B_max, s_max, Hq, Hkv, D, max_q;
     int G;                 /* Hq / Hkv                                          */
-    int variant;           /* ATTN_VARIANT_SIMT or ATTN_VARIANT_MMA             */
+    int variant;           /* ATTN_VARIANT_SIMT, _MMA or _TC                    */
     int nsplit;            /* SIMT path: KV chunks per (sequence, KV head); 0 on
                               the tensor-core path, whose split points follow
                               the balanced per-block shares                      */
@@ -153,7 +155,8 @@ int attn_plan_info(attn_plan_t plan, attn_plan_desc *desc);
 /*
  * attn_run -- one attention call, asynchronous on `stream`.
  *
- *   q      device, bf16 [T_q, Hq, D], packed and contiguous, 16-byte aligned
+ *   q      device, bf16 [T_q, Hq, D], packed and contiguous, 16-byte aligned;
+ *          readable for at least cu_q[B_max] tokens
  *   k, v   device, bf16 [T_kv, Hkv, D], packed and contiguous, 16-byte aligned;
  *          readable for at least cu_k[B_max] tokens
  *   cu_q, cu_k  device, int32, B_max + 1 entries each, 4-byte aligned:

@@ -18,7 +18,7 @@ import varlen_gqa_split_b200 as vg
 
 pytestmark = pytest.mark.gpu
 
-SIMT, MMA = vg.ATTN_VARIANT_SIMT, vg.ATTN_VARIANT_MMA
+SIMT, MMA, TC = vg.ATTN_VARIANT_SIMT, vg.ATTN_VARIANT_MMA, vg.ATTN_VARIANT_TC
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -34,7 +34,7 @@ def _gen_device(name):
 
 # ------------------------------------------------------------ the five workloads
 
-@pytest.mark.parametrize("variant", [0, SIMT, MMA])
+@pytest.mark.parametrize("variant", [0, SIMT, MMA, TC])
 @pytest.mark.parametrize("name", ["tiny", "long", "ragged"])
 def test_decode_workloads_full_parity(name, variant):
     batch = W.workload(name, gen_device=_gen_device(name))
@@ -45,7 +45,7 @@ def test_decode_workloads_full_parity(name, variant):
     compare_full(out, lse, ref_o, ref_l, cov)
 
 
-@pytest.mark.parametrize("variant", [0, SIMT])
+@pytest.mark.parametrize("variant", [0, SIMT, TC])
 def test_short_query_workload_full_parity(variant):
     batch = W.workload("shortq", gen_device="cuda")
     plan = plan_for(batch.shape, variant=variant)
@@ -140,6 +140,46 @@ def test_block_count_invariance_mma(stages, det):
         assert np.abs(o - outs[0]).max() <= 2 * ATOL_OUT
 
 
+@pytest.mark.parametrize("stages,det", [(0, 0), (0, 1), (2, 0), (3, 1)])
+def test_block_count_invariance_tc(stages, det):
+    """The tcgen05 path at 1 .. 2 x SM-count blocks on a short-query batch:
+    whole units, units cut into many parts, a unit without keys, and rows
+    that see no key under the tail-aligned causal mask (Lq > Lk)."""
+    sh = W.Shape("midq", B=5, Hq=32, Hkv=4, D=128, max_q=16, s_max=2048)
+    batch = W.make_batch(sh, [16, 3, 9, 1, 12], [2048, 700, 5, 0, 130], seed=13, gen_device="cuda")
+    ref_o, ref_l = oracle_full(batch)
+    cov = covered_rows(batch)
+    outs = []
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for ctas in (1, 2, 3, 7, 37, sms, 2 * sms):
+        plan = plan_for(sh, variant=TC, ctas=ctas, stages=stages, deterministic=det)
+        assert plan.info["ctas"] == ctas and plan.info["variant"] == TC
+        out, lse = run_gpu(plan, batch, extra_q_rows=2)
+        compare_full(out, lse, ref_o, ref_l, cov)
+        outs.append(out.float().numpy()[:len(cov)][cov])
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= 2 * ATOL_OUT
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,max_q", [(64, 4, 128, 8), (24, 4, 64, 5), (12, 12, 128, 128),
+                                            (16, 2, 64, 16), (40, 8, 128, 3)])
+def test_tc_row_layouts(Hq, Hkv, D, max_q):
+    """Query boxes of G heads x max_q tokens for several G (odd ones
+    included), both head dims, and the 128-row limit (G * max_q = 128)."""
+    rng = np.random.default_rng(Hq * 7 + max_q)
+    B = 9
+    lq = rng.integers(1, max_q, B, endpoint=True)
+    lk = np.array([rng.integers(0, 700) for _ in lq])
+    lk[0], lq[0] = 0, max_q
+    lk[1] = max(1, int(lq[1]) - 1)
+    sh = W.Shape("rows", B=B + 1, Hq=Hq, Hkv=Hkv, D=D, max_q=max_q, s_max=700)
+    batch = W.make_batch(sh, lq, lk, seed=21, gen_device="cuda")
+    plan = plan_for(sh, variant=TC, ctas=11)
+    out, lse = run_gpu(plan, batch, extra_q_rows=3)
+    ref_o, ref_l = oracle_full(batch)
+    compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
+
+
 def test_variants_agree():
     batch = W.workload("ragged", gen_device="cuda")
     a, la = run_gpu(plan_for(batch.shape, variant=SIMT), batch)
@@ -153,7 +193,7 @@ def test_variants_agree():
     assert np.abs(l1[fin] - l2[fin]).max() <= 2 * ATOL_LSE
 
 
-@pytest.mark.parametrize("kw", [{"deterministic": 1},
+@pytest.mark.parametrize("kw", [{"deterministic": 1}, {"variant": TC, "deterministic": 1},
                                 {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_FUSED},
                                 {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_KERNEL}])
 def test_repeat_runs_bitwise_equal(kw):
@@ -194,7 +234,7 @@ def _packed_cases(B, values):
     return lq, lk
 
 
-@pytest.mark.parametrize("variant", [SIMT, MMA])
+@pytest.mark.parametrize("variant", [SIMT, MMA, TC])
 def test_exhaustive_small_lengths_placement(variant):
     """Every (Lq, Lk) combination with lengths in [0, 4] for 3 sequences (the
     exhaustive method of TransformerEngine PR #24, section Equivalence), packed
@@ -214,7 +254,9 @@ def test_exhaustive_small_lengths_placement(variant):
                                 {"variant": SIMT, "nsplit": 3, "combine": vg.ATTN_COMBINE_KERNEL},
                                 {"variant": MMA, "ctas": 1}, {"variant": MMA, "ctas": 5},
                                 {"variant": MMA, "ctas": 64}, {"variant": MMA},
-                                {"variant": MMA, "ctas": 64, "deterministic": 1}])
+                                {"variant": MMA, "ctas": 64, "deterministic": 1},
+                                {"variant": TC, "ctas": 1}, {"variant": TC, "ctas": 5}, {"variant": TC},
+                                {"variant": TC, "ctas": 64, "deterministic": 1}])
 def test_ragged_multi_tile_placement(kw):
     """Lengths spanning several 64-key tiles, units cut across blocks, short
     sequences whose tile starts before the buffer (negative TMA
@@ -234,7 +276,7 @@ def test_ragged_multi_tile_placement(kw):
     compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
 
 
-@pytest.mark.parametrize("variant", [SIMT, MMA])
+@pytest.mark.parametrize("variant", [SIMT, MMA, TC])
 def test_single_key_returns_v_exactly(variant):
     sh = W.Shape("one", B=5, Hq=8, Hkv=2, D=128, max_q=1, s_max=64)
     batch = W.make_batch(sh, [1] * 5, [1] * 5, seed=2, gen_device="cuda")
@@ -245,7 +287,7 @@ def test_single_key_returns_v_exactly(variant):
     assert torch.equal(out.view(torch.int16), want.view(torch.int16))
 
 
-@pytest.mark.parametrize("variant", [SIMT, MMA])
+@pytest.mark.parametrize("variant", [SIMT, MMA, TC])
 def test_large_magnitude_scores(variant):
     sh = W.Shape("big", B=2, Hq=8, Hkv=1, D=128, max_q=1, s_max=2048)
     batch = W.make_batch(sh, [1, 1], [2048, 513], seed=4, gen_device="cuda")
@@ -264,14 +306,15 @@ def test_plan_choices_follow_the_split_rule():
     assert ragged_simt.info["nsplit"] == 1          # B * Hkv = 512 blocks already fill the SMs
     assert ragged_simt.info["scratch_bytes"] <= 1024
     sq = plan_for(W.SHAPES["shortq"])
-    assert sq.info["variant"] == SIMT
+    assert sq.info["variant"] == TC and sq.info["rows_per_block"] == 128
 
 
 # ------------------------------------------------------------ errors
 
-def test_device_side_errors_are_flagged_and_rows_untouched():
+@pytest.mark.parametrize("variant", [0, TC])
+def test_device_side_errors_are_flagged_and_rows_untouched(variant):
     sh = W.Shape("err", B=3, Hq=8, Hkv=2, D=128, max_q=1, s_max=64)
-    plan = plan_for(sh)
+    plan = plan_for(sh, variant=variant)
     g = W.make_generator(1, "cuda")
     T = 200
     q = W.bf16_normal((T, sh.Hq, sh.D), g, "cuda")
@@ -318,7 +361,9 @@ def test_host_side_errors_launch_nothing():
     with pytest.raises(vg.AttnError):
         vg.Plan(1, 64, 4, 1, 96, 1)                         # unsupported head dim
     with pytest.raises(vg.AttnError):
-        vg.Plan(1, 64, 64, 8, 128, 4, variant=MMA)         # 32 rows > tensor-core path limit
+        vg.Plan(1, 64, 64, 8, 128, 4, variant=MMA)         # 32 rows > warp-MMA path limit
+    with pytest.raises(vg.AttnError):
+        vg.Plan(1, 64, 64, 8, 128, 17, variant=TC)         # 136 rows > tcgen05 path limit
     with pytest.raises(vg.AttnError):
         vg.Plan(1, 64, 8, 1, 128, 1, variant=MMA, nsplit=2)  # split count belongs to the SIMT grid
     handle = plan.handle

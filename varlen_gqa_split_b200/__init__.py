@@ -9,9 +9,9 @@ The compute runs in libvgqa.so (C ABI: include/varlen_gqa.h); this package
 only marshals torch tensors into it.
 """
 from ._binding import (ATTN_COMBINE_AUTO, ATTN_COMBINE_FUSED, ATTN_COMBINE_KERNEL, ATTN_DEV_ERR_K_TOO_LONG, ATTN_DEV_ERR_OFFSETS, ATTN_DEV_ERR_Q_TOO_LONG,
-                       ATTN_DEV_ERR_TIMEOUT, ATTN_VARIANT_AUTO, ATTN_VARIANT_MMA, ATTN_VARIANT_SIMT,
+                       ATTN_DEV_ERR_TIMEOUT, ATTN_VARIANT_AUTO, ATTN_VARIANT_MMA, ATTN_VARIANT_SIMT, ATTN_VARIANT_TC,
                        AttnError, Plan, lib, strerror)
 
 __all__ = ["ATTN_COMBINE_AUTO", "ATTN_COMBINE_FUSED", "ATTN_COMBINE_KERNEL", "Plan", "AttnError", "lib", "strerror", "ATTN_VARIANT_AUTO", "ATTN_VARIANT_SIMT",
-           "ATTN_VARIANT_MMA", "ATTN_DEV_ERR_OFFSETS", "ATTN_DEV_ERR_Q_TOO_LONG",
+           "ATTN_VARIANT_MMA", "ATTN_VARIANT_TC", "ATTN_DEV_ERR_OFFSETS", "ATTN_DEV_ERR_Q_TOO_LONG",
            "ATTN_DEV_ERR_K_TOO_LONG", "ATTN_DEV_ERR_TIMEOUT"]

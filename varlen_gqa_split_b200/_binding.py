@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libvgqa.so")
 
 ATTN_OK = 0
-ATTN_VARIANT_AUTO, ATTN_VARIANT_SIMT, ATTN_VARIANT_MMA = 0, 1, 2
+ATTN_VARIANT_AUTO, ATTN_VARIANT_SIMT, ATTN_VARIANT_MMA, ATTN_VARIANT_TC = 0, 1, 2, 3
 ATTN_COMBINE_AUTO, ATTN_COMBINE_KERNEL, ATTN_COMBINE_FUSED = 0, 1, 2
 ATTN_DEV_ERR_OFFSETS = 0x1
 ATTN_DEV_ERR_Q_TOO_LONG = 0x2

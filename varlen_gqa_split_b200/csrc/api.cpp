@@ -76,6 +76,21 @@ int encode_kv_map(CUtensorMap *map, const void *base, int Hkv, int D, int block_
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
 }
 
+// [T, Hq, D] bf16, box = 64 elements x G heads x max_q tokens: one unit's
+// query rows (token-major, heads inner) as the tcgen05 kernel's A operand.
+// Loads are right-aligned to the sequence's last query token, so, as for K/V,
+// the token extent is left open.
+int encode_q_map(CUtensorMap *map, const void *base, int Hq, int D, int G, int max_q) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)0x7fffffff};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)max_q};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned(const void *ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
@@ -129,9 +144,16 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     d.G = Hq / Hkv;
     d.num_sms = sms;
 
-    int variant = o && o->variant ? o->variant : (rows <= 16 ? ATTN_VARIANT_MMA : ATTN_VARIANT_SIMT);
-    if (variant != ATTN_VARIANT_MMA && variant != ATTN_VARIANT_SIMT) return ATTN_E_INVALID_ARG;
+    // warp-MMA kernel up to 16 query rows per KV head (the rows ride on the
+    // MMA's n8 side), tcgen05 kernel up to 128 (the rows are the M = 128
+    // side), CUDA cores beyond
+    int variant = o && o->variant ? o->variant
+                                  : (rows <= 16 ? ATTN_VARIANT_MMA
+                                                : (rows <= tc_rows() ? ATTN_VARIANT_TC : ATTN_VARIANT_SIMT));
+    if (variant != ATTN_VARIANT_MMA && variant != ATTN_VARIANT_SIMT && variant != ATTN_VARIANT_TC)
+        return ATTN_E_INVALID_ARG;
     if (variant == ATTN_VARIANT_MMA && rows > 16) return ATTN_E_UNSUPPORTED;
+    if (variant == ATTN_VARIANT_TC && rows > tc_rows()) return ATTN_E_UNSUPPORTED;
     if (o && o->block_n && o->block_n != 64) return ATTN_E_UNSUPPORTED;
     if (o && (o->nsplit < 0 || o->stages < 0 || o->ctas < 0)) return ATTN_E_INVALID_ARG;
     if (o && o->combine && o->combine != ATTN_COMBINE_KERNEL && o->combine != ATTN_COMBINE_FUSED)
@@ -142,11 +164,12 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     int NT = 1;
     size_t n_ticket = 0, n_part = 0, part_rows = 0;
     int merge_bytes = 0;
-    if (variant == ATTN_VARIANT_MMA) {
+    if (variant == ATTN_VARIANT_MMA || variant == ATTN_VARIANT_TC) {
         // persistent: about one block per SM, each with a deep load ring; the
         // split points follow the balanced per-block shares (nsplit and chunk
         // do not apply) and the slot-parallel combine kernel merges cut units
         if (o && (o->nsplit || o->combine == ATTN_COMBINE_FUSED)) return ATTN_E_UNSUPPORTED;
+        const bool tcv = variant == ATTN_VARIANT_TC;
         NT = rows <= 8 ? 1 : 2;
         d.block_n = mma_block_n();
         const long long max_tiles = (long long)B_max * Hkv * tiles_max;
@@ -154,15 +177,16 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         ctas = std::min<long long>(ctas, std::max(1LL, max_tiles));
         ctas = std::min<long long>(ctas, 65535);
         d.ctas = (int)ctas;
-        const size_t fixed = mma_smem_bytes(D, NT, 0, d.ctas);
-        int stages = o && o->stages ? o->stages : (int)((smem_block - fixed) / mma_stage_bytes(D));
+        auto smem_of = [&](int st) { return tcv ? tc_smem_bytes(D, st) : mma_smem_bytes(D, NT, st, d.ctas); };
+        const size_t stage_bytes = tcv ? tc_stage_bytes(D) : mma_stage_bytes(D);
+        int stages = o && o->stages ? o->stages : (int)((smem_block - smem_of(0)) / stage_bytes);
         stages = std::min(stages, 8);
-        if (stages < 2 || mma_smem_bytes(D, NT, stages, d.ctas) > (size_t)smem_block) return ATTN_E_INVALID_ARG;
+        if (stages < 2 || smem_of(stages) > (size_t)smem_block) return ATTN_E_INVALID_ARG;
         d.stages = stages;
-        d.rows_per_block = 8 * NT;
+        d.rows_per_block = tcv ? tc_rows() : 8 * NT;
         d.row_tiles = 1;
-        d.smem_bytes = (int)mma_smem_bytes(D, NT, stages, d.ctas);
-        merge_bytes = (int)mma_merge_bytes(D, NT, d.ctas);
+        d.smem_bytes = (int)smem_of(stages);
+        merge_bytes = tcv ? 0 : (int)mma_merge_bytes(D, NT, d.ctas);
         d.nsplit = 0;
         d.chunk = 0;
         d.grid_x = d.ctas;
@@ -174,7 +198,8 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         n_ticket = 3 * (size_t)B_max * Hkv;  // per cut unit: tile claims (64-bit), part count
         n_part = 2 * (size_t)d.ctas;       // two partial slots per block
         part_rows = d.rows_per_block;
-        if (mma_prepare(D, NT, stages, d.ctas) != cudaSuccess) return ATTN_E_CUDA;
+        if ((tcv ? tc_prepare(D, stages, d.ctas) : mma_prepare(D, NT, stages, d.ctas)) != cudaSuccess)
+            return ATTN_E_CUDA;
     } else {
         if (o && o->ctas) return ATTN_E_UNSUPPORTED;
         d.deterministic = 1;                 // fixed grid, fixed merge order
@@ -253,7 +278,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         std::lock_guard<std::mutex> lk(g_mu);
         g_plans.insert(p);
     }
-    if (variant == ATTN_VARIANT_MMA) {
+    if (variant == ATTN_VARIANT_MMA || variant == ATTN_VARIANT_TC) {
         int rc = get_encoder();
         if (rc != ATTN_OK) {
             attn_destroy(p);
@@ -330,7 +355,9 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
     p.fused = d.combine == ATTN_COMBINE_FUSED;
     p.merge_bytes = plan->merge_bytes;
     p.ctas_max = d.ctas;
-    p.dynamic = d.variant == ATTN_VARIANT_MMA && !d.deterministic;
+    const bool persistent = d.variant == ATTN_VARIANT_MMA || d.variant == ATTN_VARIANT_TC;
+    p.dynamic = persistent && !d.deterministic;
+    p.done_per_part = d.variant == ATTN_VARIANT_TC ? tc_parts_per_block() : 1;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(d.grid_x, d.grid_y, d.grid_z);
@@ -341,6 +368,13 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
             encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n) != ATTN_OK)
             return ATTN_E_CUDA;
         e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, d.ctas, s);
+    } else if (d.variant == ATTN_VARIANT_TC) {
+        CUtensorMap tm_q, tm_k, tm_v;
+        if (encode_q_map(&tm_q, q, d.Hq, d.D, d.G, d.max_q) != ATTN_OK ||
+            encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n) != ATTN_OK ||
+            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n) != ATTN_OK)
+            return ATTN_E_CUDA;
+        e = launch_split_tc(p, tm_q, tm_k, tm_v, d.stages, d.ctas, s);
     } else {
         e = launch_split_simt(p, grid, s);
     }

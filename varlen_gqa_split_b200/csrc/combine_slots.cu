@@ -1,0 +1,199 @@
+// combine_slots.cu -- log-sum-exp merge of the partials written by the
+// persistent tensor-core split kernels (the partial-slot layout of
+// schedule.cuh: slot 2c holds block c's first cut unit, slot 2c + 1 its last;
+// a slot holds rows_per_block rows of D fp32 values plus (m, l) per row, m in
+// base-2 units of the scaled scores).
+//
+// The merge is the one the split-KV method ends with (magik.net "Wiring
+// Split-K Dispatch into a Custom CUDA Attention Kernel", section "The
+// Message"; AstrAI commit log, split-KV commit): with M = max m_s over the
+// parts that saw keys, L = sum l_s 2^(m_s - M), out = sum O_s 2^(m_s - M) / L
+// and lse = (M + log2 L) ln 2; no part with keys gives out = 0, lse = -inf.
+//
+// One block per partial slot, launched as a programmatic dependent of the
+// split kernel.  It recomputes the schedule from cu_seqlens while the split
+// kernel runs, waits only for the parts of its own unit, and merges one
+// column slice of it: the n blocks of a cut unit merge it together, each
+// reading 1/n of the partial data, so the merge is spread over as many SMs as
+// wrote it (one SM can pull only a few tens of GB/s from L2, too little to
+// merge a unit alone).
+#include "common.cuh"
+#include "kernels.h"
+#include "schedule.cuh"
+
+namespace vgqa {
+
+namespace {
+
+using namespace sched;
+
+// Combine: block 2c + k merges slice (c - c_first) of the unit block c cut at
+// its start (k = 0) or end (k = 1), if any.  The block is launched as a
+// programmatic dependent of the split kernel, so it computes the schedule
+// while the split kernel streams; it then waits (bounded) only for the n parts
+// of its own unit, whose writers each add 1 (release) to the unit's count, so
+// a unit is merged as soon as its last part lands rather than when the whole
+// split grid ends.  After merging, each of the unit's n combine blocks adds 1
+// again; the one that brings the count to 2n resets it for the next call.
+template <int D>
+__global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, const int C) {
+    constexpr int kCols = D / 4;
+    constexpr int kT = 128;
+    constexpr int kBatch = 12;             // loads in flight per thread (register budget)
+    extern __shared__ __align__(16) uint8_t csm[];
+    __shared__ long long scan[8];
+    __shared__ long long first[3];
+    __shared__ int ok_flag;
+    const int tid = threadIdx.x;
+    const int c = blockIdx.x >> 1, k = blockIdx.x & 1;
+    const long long ROWS = p.rows_per_block;     // rows of one partial slot
+    // the next call's split kernel may launch now; it waits for this grid to
+    // complete before it reads anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    Share sh;
+    if (!block_share(p, c, C, tid, kT, false, scan, first, sh)) return;
+    SegWalker wk;
+    wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
+    Segment seg;
+    wk.next(p, seg);
+    if (k == 1) {                                 // the block's last unit, when it has two or more
+        int nseg = 1;
+        while (wk.next(p, seg)) ++nseg;
+        if (nseg == 1) return;
+    }
+    if (seg.t0 == 0 && seg.t1 == seg.s.tpu) return;   // whole unit: written by the split kernel
+    const long long T = sh.T;
+    const int Ce = sh.Ce;
+    const int c_first = block_of(seg.Pu, T, Ce);
+    const int n = block_of(seg.Pu + seg.s.tpu - 1, T, Ce) - c_first + 1;
+    const int G = p.G, R = G * seg.s.Lq;
+    const int items = R * kCols;
+    const int per = (items + n - 1) / n;
+    const int it_lo = min(items, (c - c_first) * per), it_hi = min(items, it_lo + per);
+    const long long u = (long long)seg.b * p.Hkv + seg.hk;
+
+    int *slots = reinterpret_cast<int *>(csm);                         // [n]
+    for (int j = tid; j < n; j += kT) slots[j] = slot_of(c_first + j, seg.Pu, T, Ce);
+
+    // wait for the unit's n parts, each published by done_per_part release
+    // adds (the acquire pairs with them)
+    const uint32_t parts_done = (uint32_t)(n * p.done_per_part);
+    if (tid == 0) {
+        int ok = 1;
+        if (ld_acquire_gpu(p.done + u) < parts_done) {
+            const unsigned long long t0 = globaltimer();
+            while (ld_acquire_gpu(p.done + u) < parts_done) {
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(256);
+            }
+        }
+        ok_flag = ok;
+        if (ok && c == c_first) p.claim[u] = 0ull;                      // claims, next call
+    }
+    __syncthreads();
+    if (!ok_flag) return;
+
+    // two threads per item (row, 4 columns), each merging every other part
+    // with a running max, kBatch loads in flight; the pair then combines
+    const int n_work = 2 * (it_hi - it_lo);
+    for (int base = 0; base < n_work; base += kT) {
+        const int w = base + tid;
+        const bool valid = w < n_work;
+        const int it = it_lo + (valid ? w >> 1 : 0), half = w & 1;
+        const int r = it / kCols, d4 = (it % kCols) * 4;
+        float M = -INFINITY, L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) {
+            for (int j0 = half; j0 < n; j0 += 2 * kBatch) {
+                float2 ml[kBatch];
+                float4 o[kBatch];
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    const int j = j0 + 2 * q;
+                    if (j < n) {
+                        const long long sl = slots[j];
+                        ml[q] = __ldcg(p.ml_part + sl * ROWS + r);
+                        o[q] = __ldcg(reinterpret_cast<const float4 *>(p.o_part + (sl * ROWS + r) * D + d4));
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    if (j0 + 2 * q < n && ml[q].y > 0.f) {
+                        const float Mn = fmaxf(M, ml[q].x);
+                        const float a = ex2(M - Mn), wq = ex2(ml[q].x - Mn);   // ex2(-inf) = 0
+                        acc.x = fmaf(acc.x, a, wq * o[q].x);
+                        acc.y = fmaf(acc.y, a, wq * o[q].y);
+                        acc.z = fmaf(acc.z, a, wq * o[q].z);
+                        acc.w = fmaf(acc.w, a, wq * o[q].w);
+                        L = fmaf(L, a, wq * ml[q].y);
+                        M = Mn;
+                    }
+                }
+            }
+        }
+        // combine the pair (adjacent lanes)
+        const float M2 = __shfl_xor_sync(0xffffffffu, M, 1);
+        const float L2 = __shfl_xor_sync(0xffffffffu, L, 1);
+        float4 a2;
+        a2.x = __shfl_xor_sync(0xffffffffu, acc.x, 1);
+        a2.y = __shfl_xor_sync(0xffffffffu, acc.y, 1);
+        a2.z = __shfl_xor_sync(0xffffffffu, acc.z, 1);
+        a2.w = __shfl_xor_sync(0xffffffffu, acc.w, 1);
+        if (valid && half == 0) {
+            const float Mt = fmaxf(M, M2);
+            const float Mref = Mt == -INFINITY ? 0.f : Mt;
+            const float s1 = ex2(M - Mref), s2 = ex2(M2 - Mref);
+            const float Lt = L * s1 + L2 * s2;
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+            const int qi = r / G, h = seg.hk * G + r % G;
+            const long long tok = seg.s.q0 + qi;
+            uint2 pk;
+            pk.x = pack_bf16x2((acc.x * s1 + a2.x * s2) * inv, (acc.y * s1 + a2.y * s2) * inv);
+            pk.y = pack_bf16x2((acc.z * s1 + a2.z * s2) * inv, (acc.w * s1 + a2.w * s2) * inv);
+            *reinterpret_cast<uint2 *>(p.out + (tok * p.Hq + h) * D + d4) = pk;
+            if (d4 == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
+        }
+    }
+    __syncthreads();
+    // every combine block of the unit has seen its n parts once each of the
+    // n blocks has added 1 more: the last one resets the count
+    if (tid == 0 && atomicAdd(p.done + u, 1u) == parts_done + (uint32_t)(n - 1)) p.done[u] = 0u;
+}
+
+
+
+}  // namespace
+
+size_t combine_slots_smem(int ctas) { return (size_t)((ctas + 3) & ~3) * 4; }
+
+cudaError_t combine_slots_prepare(int D, int ctas) {
+    void *fn = D == 64 ? reinterpret_cast<void *>(combine_slots_kernel<64>)
+                       : reinterpret_cast<void *>(combine_slots_kernel<128>);
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)combine_slots_smem(ctas));
+}
+
+cudaError_t launch_combine_slots(const Params &p, int ctas, cudaStream_t stream) {
+    // launched as a programmatic dependent: its blocks may start (and compute
+    // the schedule) before the split kernel has finished
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * ctas);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = combine_slots_smem(ctas);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *fn = p.D == 64 ? reinterpret_cast<void *>(combine_slots_kernel<64>)
+                         : reinterpret_cast<void *>(combine_slots_kernel<128>);
+    void *args[] = {const_cast<Params *>(&p), &ctas};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+}  // namespace vgqa

@@ -28,7 +28,23 @@ cudaError_t mma_prepare(int D, int NT, int stages, int ctas);
 cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUtensorMap &tm_v, int NT,
                              int stages, int ctas, cudaStream_t stream);
 
-// log-sum-exp merge of the split partials
+// Persistent TMA-fed tcgen05 split kernel (accumulators in tensor memory),
+// up to tc_rows() query rows per KV head
+size_t tc_stage_bytes(int D);
+size_t tc_smem_bytes(int D, int stages);
+int tc_rows();
+int tc_parts_per_block();
+cudaError_t tc_prepare(int D, int stages, int ctas);
+cudaError_t launch_split_tc(const Params &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                            const CUtensorMap &tm_v, int stages, int ctas, cudaStream_t stream);
+
+// log-sum-exp merge of the persistent kernels' partial slots (2 * ctas
+// blocks, launched as a programmatic dependent of the split kernel)
+size_t combine_slots_smem(int ctas);
+cudaError_t combine_slots_prepare(int D, int ctas);
+cudaError_t launch_combine_slots(const Params &p, int ctas, cudaStream_t stream);
+
+// log-sum-exp merge of the CUDA-core kernel's dense [.., nsplit] partials
 int combine_blocks(const Params &p);
 cudaError_t launch_combine(const Params &p, cudaStream_t stream);
 

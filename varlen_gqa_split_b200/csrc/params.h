@@ -32,6 +32,7 @@ struct Params {
     int merge_bytes;           // tensor-core path: shared bytes of the merge area
     int ctas_max;              // tensor-core path: blocks of the launch (merge table size)
     int dynamic;               // tensor-core path: blocks sharing a cut unit claim its tiles
+    int done_per_part;         // tensor-core path: releases on `done` per written part
 };
 
 }  // namespace vgqa

@@ -1,0 +1,308 @@
+// schedule.cuh -- the persistent split-KV schedule shared by the tensor-core
+// split kernels and the slot combine kernel (device code, internal).
+//
+// The work is the flattened sequence of 64-key tiles of every unit
+// u = (sequence b, KV head hk), in order of b then hk; a unit with queries but
+// no keys counts as one (empty) tile so that it still gets its defined output.
+// Each of the C blocks (C fixed by the plan, about one per SM) takes the
+// contiguous, equal share [c*T/C, (c+1)*T/C) of the T tiles, computed on the
+// device from cu_seqlens at the start of every call -- no host round trip and
+// no dead blocks, whatever the lengths are.  A unit that lies inside one
+// block's share is finished there and written directly; a unit cut by share
+// boundaries is split across consecutive blocks, each of which emits one
+// unnormalised (O, m, l) partial.  A block emits at most two partials (the
+// units cut by its two boundaries), into slots 2c and 2c + 1.  This is split-KV
+// flash-decoding with the split points placed where the device can balance
+// them (AstrAI commit log for csrc/kernels/gqa_decode_attn.cu, split-KV
+// commit; cudnn-frontend issue #552 "frost(sdpa): THD execute host
+// round-trip", sections Context and Proposal to evaluate: device lengths, no
+// host totals).
+#pragma once
+
+#include "common.cuh"
+
+namespace vgqa {
+namespace sched {
+
+constexpr int kBN = 64;                   // keys per tile
+constexpr int kClaim = 2;                 // tiles per claim on a shared unit's counter
+
+// tiles of one unit of sequence b: 0 if the sequence is skipped (no query
+// rows, or lengths outside the plan), else max(1, ceil(Lk / 64))
+__device__ __forceinline__ int unit_tiles(int Lq, int Lk, bool ok) {
+    if (!ok || Lq <= 0) return 0;
+    return Lk > 0 ? (Lk + kBN - 1) / kBN : 1;
+}
+
+struct SeqLen {
+    int q0, Lq, k0, Lk, tpu;
+};
+
+__device__ __forceinline__ SeqLen seq_len(const Params &p, int b, bool report) {
+    SeqLen s;
+    const bool ok = load_lengths(p, b, report, s.q0, s.Lq, s.k0, s.Lk);
+    s.tpu = unit_tiles(s.Lq, s.Lk, ok);
+    return s;
+}
+
+// One stretch of a unit inside a block's share.
+struct Segment {
+    int b, hk;
+    SeqLen s;
+    int t0, t1;           // tiles [t0, t1) of the unit's tpu tiles
+    long long Pu;         // global index of the unit's first tile
+};
+
+// Walks a block's share [g, hi) of the flattened tile space unit by unit.
+struct SegWalker {
+    int b, hk;
+    SeqLen s;
+    long long pb;         // global index of tile 0 of (b, hk = 0)
+    long long g, hi;
+
+    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi_) {
+        b = b_first;
+        pb = pb_first;
+        s = seq_len(p, b, false);
+        hk = (int)((lo - pb) / s.tpu);
+        g = lo;
+        hi = hi_;
+    }
+
+    __device__ bool next(const Params &p, Segment &seg) {
+        if (g >= hi) return false;
+        const long long Pu = pb + (long long)hk * s.tpu;
+        seg.b = b;
+        seg.hk = hk;
+        seg.s = s;
+        seg.Pu = Pu;
+        seg.t0 = (int)(g - Pu);
+        const long long end = min(hi, Pu + s.tpu);
+        seg.t1 = (int)(end - Pu);
+        g = end;
+        if (g < hi && ++hk == p.Hkv) {
+            // next sequence with work; the share ends before the tiles do, so
+            // one exists (the bound only guards against reading past cu)
+            pb += (long long)p.Hkv * s.tpu;
+            hk = 0;
+            do {
+                if (++b >= p.B_max) {
+                    g = hi;
+                    break;
+                }
+                s = seq_len(p, b, false);
+            } while (s.tpu == 0);
+        }
+        return true;
+    }
+};
+
+// A block's units in processing order: the units that lie inside its share
+// (streamed and written by this block alone) first, then the unit cut at the
+// share's start (role 1, partial slot 2c), then the unit cut at its end
+// (role 2, slot 2c + 1).  Cut units come last so that every block sharing one
+// reaches it near the end of its own work, where run-time balancing can even
+// out the blocks' finishing times without delaying any block's own units.
+struct OrderedWalker {
+    SegWalker wk;
+    Segment first_cut, last_cut;
+    bool has_first, has_last;
+    int phase;            // 0: inside units, 1: the start-cut unit, 2: the end-cut unit, 3: done
+
+    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi) {
+        wk.init(p, b_first, pb_first, lo, hi);
+        wk_lo = lo;
+        has_first = has_last = false;
+        phase = 0;
+    }
+
+    // role: 0 = unit inside the share, 1 = cut at the share's start, 2 = cut at its end
+    __device__ bool next(const Params &p, Segment &seg, int &role) {
+        if (phase == 0) {
+            Segment s;
+            while (true) {
+                const long long g0 = wk.g;
+                if (!wk.next(p, s)) break;
+                const bool whole = s.t0 == 0 && s.t1 == s.s.tpu;
+                if (whole) {
+                    seg = s;
+                    role = 0;
+                    return true;
+                }
+                if (g0 == wk_lo) {
+                    first_cut = s;
+                    has_first = true;
+                } else {
+                    last_cut = s;
+                    has_last = true;
+                }
+            }
+            phase = 1;
+        }
+        if (phase == 1) {
+            phase = 2;
+            if (has_first) {
+                seg = first_cut;
+                role = 1;
+                return true;
+            }
+        }
+        if (phase == 2) {
+            phase = 3;
+            if (has_last) {
+                seg = last_cut;
+                role = 2;
+                return true;
+            }
+        }
+        return false;
+    }
+    long long wk_lo;
+};
+
+// block whose share [c*T/C, (c+1)*T/C) holds global tile t
+__device__ __forceinline__ int block_of(long long t, long long T, int C) {
+    return (int)(((t + 1) * C - 1) / T);
+}
+__device__ __forceinline__ long long share_start(int c, long long T, int C) {
+    return (long long)c * T / C;
+}
+
+// Partial slot of block c for the unit whose first tile is Pu: a block's first
+// unit uses slot 2c, its last (cut) unit slot 2c + 1.
+__device__ __forceinline__ int slot_of(int c, long long Pu, long long T, int C) {
+    return share_start(c, T, C) < Pu ? 2 * c + 1 : 2 * c;
+}
+
+// The block's share of the flattened tile space, computed by all `nthreads`
+// threads of the block from cu_seqlens.  Each thread weighs a contiguous run of
+// sequences; a scan of the run totals gives the tile prefix, the total T and
+// the share; the thread whose run holds the share's first tile finds its unit.
+// scan: 8 long long, first: 3 long long of shared memory.
+struct Share {
+    long long T, lo, hi, pb_first;
+    int Ce, b_first;
+};
+
+__device__ __forceinline__ bool block_share(const Params &p, int c, int C, int tid, int nthreads, bool report,
+                            long long *scan, long long *first, Share &sh) {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int per = (p.B_max + nthreads - 1) / nthreads;
+    const int b_lo = min(p.B_max, tid * per), b_hi = min(p.B_max, b_lo + per);
+    long long my = 0;
+    for (int b = b_lo; b < b_hi; ++b) my += (long long)p.Hkv * seq_len(p, b, report).tpu;
+    long long incl = my;                                    // warp-inclusive scan
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) scan[warp] = incl;
+    if (tid == 0) first[0] = -1;
+    __syncthreads();
+    if (tid == 0) {
+        long long run = 0;
+        for (int w = 0; w < nthreads / 32; ++w) {
+            const long long x = scan[w];
+            scan[w] = run;
+            run += x;
+        }
+        first[2] = run;
+    }
+    __syncthreads();
+    sh.T = first[2];
+    const long long my_start = incl - my + scan[warp];      // tiles before this thread's run
+    // with fewer tiles than blocks only the first T blocks take a share, so
+    // that every share between two blocks of a cut unit holds a tile of it
+    sh.Ce = (int)min((long long)C, sh.T);
+    if (c >= sh.Ce) return false;                           // no tiles for this block
+    sh.lo = share_start(c, sh.T, sh.Ce);
+    sh.hi = share_start(c + 1, sh.T, sh.Ce);
+    long long pb = my_start;
+    if (sh.lo >= pb && sh.lo < pb + my) {
+        for (int b = b_lo; b < b_hi; ++b) {
+            const long long w = (long long)p.Hkv * seq_len(p, b, false).tpu;
+            if (sh.lo < pb + w) {
+                first[0] = b;
+                first[1] = pb;
+                break;
+            }
+            pb += w;
+        }
+    }
+    __syncthreads();
+    sh.b_first = (int)first[0];
+    sh.pb_first = first[1];
+    return sh.b_first >= 0;                                 // always when lo < T
+}
+
+// The block's tiles in the order its producer loads them.  For every segment
+// of the block (OrderedWalker order) begin(seg, role) runs once, then
+// tile(seg, t, last) for each tile t of the unit the block takes -- `last`
+// marks the block's final tile of that unit -- or none(seg) if it takes none.
+// A unit inside the share, and every unit in deterministic mode, is taken as
+// the static share gives it.  In the run-time balanced mode the blocks that
+// share a cut unit consume it from both ends through one packed counter per
+// unit (front count in the high word, back count in the low word): the block
+// whose static part is the unit's front claims upward, the others downward,
+// kClaim tiles at a time with one claim in flight ahead of the tiles it feeds;
+// each claim gets the part of its range that the counter's old value shows as
+// still free.  A callback returns false to stop the walk (a wait gave up);
+// the function then returns false.
+template <class Begin, class Tile, class None>
+__device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long long pb_first, long long lo,
+                                           long long hi, Begin &&begin, Tile &&tile, None &&none) {
+    OrderedWalker wk;
+    wk.init(p, b_first, pb_first, lo, hi);
+    Segment seg;
+    int role;
+    while (wk.next(p, seg, role)) {
+        if (!begin(seg, role)) return false;
+        const int ntiles = (seg.s.Lk + kBN - 1) / kBN;
+        if (role == 0 || !p.dynamic) {
+            const int tb = role == 0 ? 0 : seg.t0, te = role == 0 ? ntiles : min(ntiles, seg.t1);
+            for (int t = tb; t < te; ++t)
+                if (!tile(seg, t, t == te - 1)) return false;
+            if (te <= tb && !none(seg)) return false;
+            continue;
+        }
+        unsigned long long *claim = p.claim + (long long)seg.b * p.Hkv + seg.hk;
+        const bool up = seg.t0 == 0;                       // static part at the unit's front
+        const unsigned long long inc = up ? ((unsigned long long)kClaim << 32) : (unsigned long long)kClaim;
+        auto range = [&](unsigned long long old, int &t_lo, int &t_hi) {
+            const int f = (int)(old >> 32), b = (int)(old & 0xffffffffu);
+            const int free_hi = ntiles - b;
+            if (up) {
+                t_lo = f;
+                t_hi = min(f + kClaim, free_hi);
+            } else {
+                t_hi = free_hi;
+                t_lo = max(free_hi - kClaim, f);
+            }
+        };
+        int a_lo, a_hi, n_lo, n_hi;
+        range(atomicAdd(claim, inc), a_lo, a_hi);
+        bool any = false;
+        while (a_lo < a_hi) {
+            // next claim in flight, unless this one already reached the far end
+            const bool more = up ? a_hi < ntiles : a_lo > 0;
+            if (more)
+                range(atomicAdd(claim, inc), n_lo, n_hi);
+            else
+                n_lo = n_hi = 0;
+            const bool final_range = !(n_lo < n_hi);
+            for (int i = 0; i < a_hi - a_lo; ++i) {
+                const int t = up ? a_lo + i : a_hi - 1 - i;
+                if (!tile(seg, t, final_range && i == a_hi - a_lo - 1)) return false;
+                any = true;
+            }
+            a_lo = n_lo;
+            a_hi = n_hi;
+        }
+        if (!any && !none(seg)) return false;
+    }
+    return true;
+}
+
+}  // namespace sched
+}  // namespace vgqa

@@ -1,23 +1,10 @@
-// split_mma.cu -- persistent TMA-fed tensor-core split-KV kernel for
-// decode-sized row counts (G * q_len <= 16 query rows per KV head), and the
-// log-sum-exp combine kernel that follows it.
+// split_mma.cu -- persistent TMA-fed warp-MMA split-KV kernel for
+// decode-sized row counts (G * q_len <= 16 query rows per KV head).
 //
-// Schedule.  The work is the flattened sequence of 64-key tiles of every unit
-// u = (sequence b, KV head hk), in order of b then hk; a unit with queries but
-// no keys counts as one (empty) tile so that it still gets its defined output.
-// Each of the C blocks (C fixed by the plan, about one per SM) takes the
-// contiguous, equal share [c*T/C, (c+1)*T/C) of the T tiles, computed on the
-// device from cu_seqlens at the start of every call -- no host round trip and
-// no dead blocks, whatever the lengths are.  A unit that lies inside one
-// block's share is finished there and written directly; a unit cut by share
-// boundaries is split across consecutive blocks, each of which emits one
-// unnormalised (O, m, l) partial.  A block emits at most two partials (the
-// units cut by its two boundaries), into slots 2c and 2c + 1.  This is split-KV
-// flash-decoding with the split points placed where the device can balance
-// them (AstrAI commit log for csrc/kernels/gqa_decode_attn.cu, split-KV
-// commit; cudnn-frontend issue #552 "frost(sdpa): THD execute host
-// round-trip", sections Context and Proposal to evaluate: device lengths, no
-// host totals).
+// The schedule (schedule.cuh): a persistent grid of about one block per SM,
+// each taking an equal contiguous share of the flattened 64-key tiles of all
+// (sequence, KV head) units; units cut by share boundaries become partials
+// that the slot combine kernel (combine_slots.cu) merges.
 //
 // Split kernel: 4 consumer warps + 1 producer warp per block.
 //
@@ -43,27 +30,20 @@
 // raw bf16 in registers (prefetched one unit ahead) and the softmax scale
 // enters in fp32 inside the exp2 argument.  At the end of a unit the four
 // warp states are merged in shared memory and written.
-//
-// Combine kernel: one block per partial slot, launched as a programmatic
-// dependent of the split kernel.  It recomputes the schedule from cu_seqlens
-// while the split kernel runs, waits only for the parts of its own unit, and
-// merges one column slice of it: the n blocks of a cut unit merge it
-// together, each reading 1/n of the partial data, so the merge is spread over
-// as many SMs as wrote it (one SM can pull only a few tens of GB/s from L2,
-// too little to merge a unit alone).
 #include "common.cuh"
 #include "kernels.h"
+#include "schedule.cuh"
 
 namespace vgqa {
 
 namespace {
 
-constexpr int kBN = 64;                   // keys per tile
+using namespace sched;
+
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr int kBarConsumers = 1;          // named barrier of the consumer warps
-constexpr int kClaim = 2;                 // tiles per claim on a shared unit's counter
 constexpr int kMetaLast = 1;              // stage flag: the block's last tile of the unit
 constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends here
 
@@ -78,215 +58,6 @@ struct MmaLayout {
 // byte offset of (row, 16-byte chunk c) inside a 128B-swizzled [rows][128 B] region
 __device__ __forceinline__ uint32_t swz(int row, int c) {
     return row * 128 + ((c ^ (row & 7)) << 4);
-}
-
-// tiles of one unit of sequence b: 0 if the sequence is skipped (no query
-// rows, or lengths outside the plan), else max(1, ceil(Lk / 64))
-__device__ __forceinline__ int unit_tiles(int Lq, int Lk, bool ok) {
-    if (!ok || Lq <= 0) return 0;
-    return Lk > 0 ? (Lk + kBN - 1) / kBN : 1;
-}
-
-struct SeqLen {
-    int q0, Lq, k0, Lk, tpu;
-};
-
-__device__ __forceinline__ SeqLen seq_len(const Params &p, int b, bool report) {
-    SeqLen s;
-    const bool ok = load_lengths(p, b, report, s.q0, s.Lq, s.k0, s.Lk);
-    s.tpu = unit_tiles(s.Lq, s.Lk, ok);
-    return s;
-}
-
-// One stretch of a unit inside a block's share.
-struct Segment {
-    int b, hk;
-    SeqLen s;
-    int t0, t1;           // tiles [t0, t1) of the unit's tpu tiles
-    long long Pu;         // global index of the unit's first tile
-};
-
-// Walks a block's share [g, hi) of the flattened tile space unit by unit.
-struct SegWalker {
-    int b, hk;
-    SeqLen s;
-    long long pb;         // global index of tile 0 of (b, hk = 0)
-    long long g, hi;
-
-    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi_) {
-        b = b_first;
-        pb = pb_first;
-        s = seq_len(p, b, false);
-        hk = (int)((lo - pb) / s.tpu);
-        g = lo;
-        hi = hi_;
-    }
-
-    __device__ bool next(const Params &p, Segment &seg) {
-        if (g >= hi) return false;
-        const long long Pu = pb + (long long)hk * s.tpu;
-        seg.b = b;
-        seg.hk = hk;
-        seg.s = s;
-        seg.Pu = Pu;
-        seg.t0 = (int)(g - Pu);
-        const long long end = min(hi, Pu + s.tpu);
-        seg.t1 = (int)(end - Pu);
-        g = end;
-        if (g < hi && ++hk == p.Hkv) {
-            // next sequence with work; the share ends before the tiles do, so
-            // one exists (the bound only guards against reading past cu)
-            pb += (long long)p.Hkv * s.tpu;
-            hk = 0;
-            do {
-                if (++b >= p.B_max) {
-                    g = hi;
-                    break;
-                }
-                s = seq_len(p, b, false);
-            } while (s.tpu == 0);
-        }
-        return true;
-    }
-};
-
-// A block's units in processing order: the units that lie inside its share
-// (streamed and written by this block alone) first, then the unit cut at the
-// share's start (role 1, partial slot 2c), then the unit cut at its end
-// (role 2, slot 2c + 1).  Cut units come last so that every block sharing one
-// reaches it near the end of its own work, where run-time balancing can even
-// out the blocks' finishing times without delaying any block's own units.
-struct OrderedWalker {
-    SegWalker wk;
-    Segment first_cut, last_cut;
-    bool has_first, has_last;
-    int phase;            // 0: inside units, 1: the start-cut unit, 2: the end-cut unit, 3: done
-
-    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi) {
-        wk.init(p, b_first, pb_first, lo, hi);
-        wk_lo = lo;
-        has_first = has_last = false;
-        phase = 0;
-    }
-
-    // role: 0 = unit inside the share, 1 = cut at the share's start, 2 = cut at its end
-    __device__ bool next(const Params &p, Segment &seg, int &role) {
-        if (phase == 0) {
-            Segment s;
-            while (true) {
-                const long long g0 = wk.g;
-                if (!wk.next(p, s)) break;
-                const bool whole = s.t0 == 0 && s.t1 == s.s.tpu;
-                if (whole) {
-                    seg = s;
-                    role = 0;
-                    return true;
-                }
-                if (g0 == wk_lo) {
-                    first_cut = s;
-                    has_first = true;
-                } else {
-                    last_cut = s;
-                    has_last = true;
-                }
-            }
-            phase = 1;
-        }
-        if (phase == 1) {
-            phase = 2;
-            if (has_first) {
-                seg = first_cut;
-                role = 1;
-                return true;
-            }
-        }
-        if (phase == 2) {
-            phase = 3;
-            if (has_last) {
-                seg = last_cut;
-                role = 2;
-                return true;
-            }
-        }
-        return false;
-    }
-    long long wk_lo;
-};
-
-// block whose share [c*T/C, (c+1)*T/C) holds global tile t
-__device__ __forceinline__ int block_of(long long t, long long T, int C) {
-    return (int)(((t + 1) * C - 1) / T);
-}
-__device__ __forceinline__ long long share_start(int c, long long T, int C) {
-    return (long long)c * T / C;
-}
-
-// Partial slot of block c for the unit whose first tile is Pu: a block's first
-// unit uses slot 2c, its last (cut) unit slot 2c + 1.
-__device__ __forceinline__ int slot_of(int c, long long Pu, long long T, int C) {
-    return share_start(c, T, C) < Pu ? 2 * c + 1 : 2 * c;
-}
-
-// The block's share of the flattened tile space, computed by all `nthreads`
-// threads of the block from cu_seqlens.  Each thread weighs a contiguous run of
-// sequences; a scan of the run totals gives the tile prefix, the total T and
-// the share; the thread whose run holds the share's first tile finds its unit.
-// scan: 8 long long, first: 3 long long of shared memory.
-struct Share {
-    long long T, lo, hi, pb_first;
-    int Ce, b_first;
-};
-
-__device__ bool block_share(const Params &p, int c, int C, int tid, int nthreads, bool report,
-                            long long *scan, long long *first, Share &sh) {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int per = (p.B_max + nthreads - 1) / nthreads;
-    const int b_lo = min(p.B_max, tid * per), b_hi = min(p.B_max, b_lo + per);
-    long long my = 0;
-    for (int b = b_lo; b < b_hi; ++b) my += (long long)p.Hkv * seq_len(p, b, report).tpu;
-    long long incl = my;                                    // warp-inclusive scan
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const long long y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-    }
-    if (lane == 31) scan[warp] = incl;
-    if (tid == 0) first[0] = -1;
-    __syncthreads();
-    if (tid == 0) {
-        long long run = 0;
-        for (int w = 0; w < nthreads / 32; ++w) {
-            const long long x = scan[w];
-            scan[w] = run;
-            run += x;
-        }
-        first[2] = run;
-    }
-    __syncthreads();
-    sh.T = first[2];
-    const long long my_start = incl - my + scan[warp];      // tiles before this thread's run
-    // with fewer tiles than blocks only the first T blocks take a share, so
-    // that every share between two blocks of a cut unit holds a tile of it
-    sh.Ce = (int)min((long long)C, sh.T);
-    if (c >= sh.Ce) return false;                           // no tiles for this block
-    sh.lo = share_start(c, sh.T, sh.Ce);
-    sh.hi = share_start(c + 1, sh.T, sh.Ce);
-    long long pb = my_start;
-    if (sh.lo >= pb && sh.lo < pb + my) {
-        for (int b = b_lo; b < b_hi; ++b) {
-            const long long w = (long long)p.Hkv * seq_len(p, b, false).tpu;
-            if (sh.lo < pb + w) {
-                first[0] = b;
-                first[1] = pb;
-                break;
-            }
-            pb += w;
-        }
-    }
-    __syncthreads();
-    sh.b_first = (int)first[0];
-    sh.pb_first = first[1];
-    return sh.b_first >= 0;                                 // always when lo < T
 }
 
 template <int D, int NT>
@@ -344,27 +115,15 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     __syncthreads();
 
     // ------------------------------------------------------------ producer
-    // Units inside this block's share are streamed whole.  A cut unit is
-    // shared with the neighbouring block(s): in the run-time balanced mode the
-    // blocks sharing it consume it from both ends through one packed counter
-    // per unit (front count in the high word, back count in the low word), the
-    // block whose static part is the unit's front claiming upward and the
-    // others downward, kClaim tiles at a time with one claim in flight ahead
-    // of the loads it feeds; each claim gets the part of its range that the
-    // counter's old value shows as still free.  In deterministic mode each
-    // block streams its static part.  Every stage carries its tile's key start
-    // and a flag in shared memory; the block's last stage of a unit is flagged
-    // (an empty stage carries the flag when the block got no tile of it).
+    // One lane feeds the ring with the block's tiles (schedule.cuh
+    // feed_tiles).  Every stage carries its tile's key start and a flag in
+    // shared memory; the block's last stage of a unit is flagged (an empty
+    // stage carries the flag when the block got no tile of it).
     if (warp == kConsumerWarps) {
         if (lane == 0) {
             const uint64_t pol = l2_evict_first();
-            OrderedWalker wk;
-            wk.init(p, b_first, pb_first, lo, hi);
-            Segment seg;
-            int role;
             int s = 0, issued = 0;
             uint32_t phase = 0;
-            bool ok = true;
             // take the next free stage; false if the wait gave up
             auto acquire = [&]() -> bool {
                 if (issued >= stages && !mbar_wait(&empty[s], phase ^ 1)) {
@@ -380,7 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                     phase ^= 1;
                 }
             };
-            auto load_tile = [&](const Segment &sg, int tile, bool last) {
+            auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
+                if (!acquire()) return false;
                 const int ks = tile * kBN;
                 const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
                 meta[s] = make_int2(ks, last ? kMetaLast : 0);
@@ -392,68 +152,18 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
 #pragma unroll
                 for (int hf = 0; hf < L::kHalves; ++hf)
                     tma_load_3d(st + L::kTileBytes + hf * L::kRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
+                advance();
+                return true;
             };
-            auto empty_stage = [&]() {                 // end of a unit without a tile
+            auto empty_stage = [&](const Segment &) -> bool {   // end of a unit without a tile
+                if (!acquire()) return false;
                 meta[s] = make_int2(0, kMetaLast | kMetaEmpty);
                 mbar_arrive(&full[s]);
+                advance();
+                return true;
             };
-            while (ok && wk.next(p, seg, role)) {
-                const int ntiles = (seg.s.Lk + kBN - 1) / kBN;
-                if (role == 0 || !p.dynamic) {
-                    const int tb = role == 0 ? 0 : seg.t0, te = role == 0 ? ntiles : min(ntiles, seg.t1);
-                    for (int t = tb; t < te; ++t) {
-                        if (!(ok = acquire())) break;
-                        load_tile(seg, t, t == te - 1);
-                        advance();
-                    }
-                    if (ok && te <= tb) {
-                        if (!(ok = acquire())) break;
-                        empty_stage();
-                        advance();
-                    }
-                    continue;
-                }
-                unsigned long long *claim = p.claim + (long long)seg.b * p.Hkv + seg.hk;
-                const bool up = seg.t0 == 0;                       // static part at the unit's front
-                const unsigned long long inc = up ? ((unsigned long long)kClaim << 32) : (unsigned long long)kClaim;
-                auto range = [&](unsigned long long old, int &t_lo, int &t_hi) {
-                    const int f = (int)(old >> 32), b = (int)(old & 0xffffffffu);
-                    const int free_hi = ntiles - b;
-                    if (up) {
-                        t_lo = f;
-                        t_hi = min(f + kClaim, free_hi);
-                    } else {
-                        t_hi = free_hi;
-                        t_lo = max(free_hi - kClaim, f);
-                    }
-                };
-                int a_lo, a_hi, n_lo, n_hi;
-                range(atomicAdd(claim, inc), a_lo, a_hi);
-                bool any = false;
-                while (ok && a_lo < a_hi) {
-                    // next claim in flight, unless this one already reached the far end
-                    const bool more = up ? a_hi < ntiles : a_lo > 0;
-                    if (more)
-                        range(atomicAdd(claim, inc), n_lo, n_hi);
-                    else
-                        n_lo = n_hi = 0;
-                    const bool final_range = !(n_lo < n_hi);
-                    for (int i = 0; i < a_hi - a_lo; ++i) {
-                        const int t = up ? a_lo + i : a_hi - 1 - i;
-                        if (!(ok = acquire())) break;
-                        load_tile(seg, t, final_range && i == a_hi - a_lo - 1);
-                        advance();
-                        any = true;
-                    }
-                    a_lo = n_lo;
-                    a_hi = n_hi;
-                }
-                if (ok && !any) {
-                    if (!(ok = acquire())) break;
-                    empty_stage();
-                    advance();
-                }
-            }
+            feed_tiles(p, b_first, pb_first, lo, hi, [](const Segment &, int) { return true; }, load_tile,
+                       empty_stage);
         }
         return;
     }
@@ -703,147 +413,6 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     }
 }
 
-// Combine: block 2c + k merges slice (c - c_first) of the unit block c cut at
-// its start (k = 0) or end (k = 1), if any.  The block is launched as a
-// programmatic dependent of the split kernel, so it computes the schedule
-// while the split kernel streams; it then waits (bounded) only for the n parts
-// of its own unit, whose writers each add 1 (release) to the unit's count, so
-// a unit is merged as soon as its last part lands rather than when the whole
-// split grid ends.  After merging, each of the unit's n combine blocks adds 1
-// again; the one that brings the count to 2n resets it for the next call.
-template <int D, int NT>
-__global__ void __launch_bounds__(128, 4) combine_mma_kernel(const Params p, const int C) {
-    constexpr int ROWS = 8 * NT;
-    constexpr int kCols = D / 4;
-    constexpr int kT = 128;
-    constexpr int kBatch = 12;             // loads in flight per thread (register budget)
-    extern __shared__ __align__(16) uint8_t csm[];
-    __shared__ long long scan[8];
-    __shared__ long long first[3];
-    __shared__ int ok_flag;
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int c = blockIdx.x >> 1, k = blockIdx.x & 1;
-    // the next call's split kernel may launch now; it waits for this grid to
-    // complete before it reads anything
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-    Share sh;
-    if (!block_share(p, c, C, tid, kT, false, scan, first, sh)) return;
-    SegWalker wk;
-    wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
-    Segment seg;
-    wk.next(p, seg);
-    if (k == 1) {                                 // the block's last unit, when it has two or more
-        int nseg = 1;
-        while (wk.next(p, seg)) ++nseg;
-        if (nseg == 1) return;
-    }
-    if (seg.t0 == 0 && seg.t1 == seg.s.tpu) return;   // whole unit: written by the split kernel
-    const long long T = sh.T;
-    const int Ce = sh.Ce;
-    const int c_first = block_of(seg.Pu, T, Ce);
-    const int n = block_of(seg.Pu + seg.s.tpu - 1, T, Ce) - c_first + 1;
-    const int G = p.G, R = G * seg.s.Lq;
-    const int items = R * kCols;
-    const int per = (items + n - 1) / n;
-    const int it_lo = min(items, (c - c_first) * per), it_hi = min(items, it_lo + per);
-    const long long u = (long long)seg.b * p.Hkv + seg.hk;
-
-    int *slots = reinterpret_cast<int *>(csm);                         // [n]
-    for (int j = tid; j < n; j += kT) slots[j] = slot_of(c_first + j, seg.Pu, T, Ce);
-
-    // wait for the unit's n parts (acquire pairs with the writers' release)
-    if (tid == 0) {
-        int ok = 1;
-        if (ld_acquire_gpu(p.done + u) < (uint32_t)n) {
-            const unsigned long long t0 = globaltimer();
-            while (ld_acquire_gpu(p.done + u) < (uint32_t)n) {
-                if (globaltimer() - t0 > kWaitLimitNs) {
-                    atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(256);
-            }
-        }
-        ok_flag = ok;
-        if (ok && c == c_first) p.claim[u] = 0ull;                      // claims, next call
-    }
-    __syncthreads();
-    if (!ok_flag) return;
-
-    // two threads per item (row, 4 columns), each merging every other part
-    // with a running max, kBatch loads in flight; the pair then combines
-    const int n_work = 2 * (it_hi - it_lo);
-    for (int base = 0; base < n_work; base += kT) {
-        const int w = base + tid;
-        const bool valid = w < n_work;
-        const int it = it_lo + (valid ? w >> 1 : 0), half = w & 1;
-        const int r = it / kCols, d4 = (it % kCols) * 4;
-        float M = -INFINITY, L = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid) {
-            for (int j0 = half; j0 < n; j0 += 2 * kBatch) {
-                float2 ml[kBatch];
-                float4 o[kBatch];
-#pragma unroll
-                for (int q = 0; q < kBatch; ++q) {
-                    const int j = j0 + 2 * q;
-                    if (j < n) {
-                        const long long sl = slots[j];
-                        ml[q] = __ldcg(p.ml_part + sl * ROWS + r);
-                        o[q] = __ldcg(reinterpret_cast<const float4 *>(p.o_part + (sl * ROWS + r) * D + d4));
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < kBatch; ++q) {
-                    if (j0 + 2 * q < n && ml[q].y > 0.f) {
-                        const float Mn = fmaxf(M, ml[q].x);
-                        const float a = ex2(M - Mn), wq = ex2(ml[q].x - Mn);   // ex2(-inf) = 0
-                        acc.x = fmaf(acc.x, a, wq * o[q].x);
-                        acc.y = fmaf(acc.y, a, wq * o[q].y);
-                        acc.z = fmaf(acc.z, a, wq * o[q].z);
-                        acc.w = fmaf(acc.w, a, wq * o[q].w);
-                        L = fmaf(L, a, wq * ml[q].y);
-                        M = Mn;
-                    }
-                }
-            }
-        }
-        // combine the pair (adjacent lanes)
-        const float M2 = __shfl_xor_sync(0xffffffffu, M, 1);
-        const float L2 = __shfl_xor_sync(0xffffffffu, L, 1);
-        float4 a2;
-        a2.x = __shfl_xor_sync(0xffffffffu, acc.x, 1);
-        a2.y = __shfl_xor_sync(0xffffffffu, acc.y, 1);
-        a2.z = __shfl_xor_sync(0xffffffffu, acc.z, 1);
-        a2.w = __shfl_xor_sync(0xffffffffu, acc.w, 1);
-        if (valid && half == 0) {
-            const float Mt = fmaxf(M, M2);
-            const float Mref = Mt == -INFINITY ? 0.f : Mt;
-            const float s1 = ex2(M - Mref), s2 = ex2(M2 - Mref);
-            const float Lt = L * s1 + L2 * s2;
-            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
-            const int qi = r / G, h = seg.hk * G + r % G;
-            const long long tok = seg.s.q0 + qi;
-            uint2 pk;
-            pk.x = pack_bf16x2((acc.x * s1 + a2.x * s2) * inv, (acc.y * s1 + a2.y * s2) * inv);
-            pk.y = pack_bf16x2((acc.z * s1 + a2.z * s2) * inv, (acc.w * s1 + a2.w * s2) * inv);
-            *reinterpret_cast<uint2 *>(p.out + (tok * p.Hq + h) * D + d4) = pk;
-            if (d4 == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
-        }
-    }
-    (void)lane;
-    __syncthreads();
-    // every combine block of the unit has seen its n parts once the count
-    // reaches 2n: the last one resets it
-    if (tid == 0 && atomicAdd(p.done + u, 1u) == (uint32_t)(2 * n - 1)) p.done[u] = 0u;
-}
-
-size_t combine_mma_smem(int /*NT*/, int ctas) {
-    return (size_t)((ctas + 3) & ~3) * 4;
-}
-
 template <int D, int NT>
 void *mma_kernel_ptr() {
     return reinterpret_cast<void *>(split_mma_kernel<D, NT>);
@@ -876,20 +445,11 @@ size_t mma_smem_bytes(int D, int NT, int stages, int ctas) {
 int mma_block_n() { return kBN; }
 int mma_threads() { return kThreads; }
 
-void *combine_pick(int D, int NT) {
-    if (D == 64)
-        return NT == 1 ? reinterpret_cast<void *>(combine_mma_kernel<64, 1>)
-                       : reinterpret_cast<void *>(combine_mma_kernel<64, 2>);
-    return NT == 1 ? reinterpret_cast<void *>(combine_mma_kernel<128, 1>)
-                   : reinterpret_cast<void *>(combine_mma_kernel<128, 2>);
-}
-
 cudaError_t mma_prepare(int D, int NT, int stages, int ctas) {
     cudaError_t e = cudaFuncSetAttribute(pick(D, NT), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)mma_smem_bytes(D, NT, stages, ctas));
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(combine_pick(D, NT), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)combine_mma_smem(NT, ctas));
+    return combine_slots_prepare(D, ctas);
 }
 
 cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUtensorMap &tm_v, int NT,
@@ -914,11 +474,7 @@ cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUt
                           const_cast<Params *>(&p), &st};
     cudaError_t e = cudaLaunchKernelExC(&cfg, pick(p.D, NT), split_args);
     if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3(2 * ctas);
-    cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = combine_mma_smem(NT, ctas);
-    void *combine_args[] = {const_cast<Params *>(&p), &ctas};
-    return cudaLaunchKernelExC(&cfg, combine_pick(p.D, NT), combine_args);
+    return launch_combine_slots(p, ctas, stream);
 }
 
 }  // namespace vgqa

@@ -1,0 +1,537 @@
+// split_tc.cu -- persistent TMA-fed split-KV kernel on the fifth-generation
+// tensor cores (tcgen05, accumulators in tensor memory) for short-query row
+// counts: up to 128 query rows (G * max_q) per KV head.
+//
+// Same schedule as the warp-MMA kernel (schedule.cuh: equal shares of the
+// flattened 64-key tiles, cut units merged by the slot combine kernel), but
+// the G query heads times the q_len query tokens of a unit form the M = 128
+// side of real tensor-core tiles (kernbench2 docs/adr-proposed commit log,
+// GQA entry: G folded into the matmul M dimension; every K/V byte is read
+// once per KV head):
+//     S [128 rows x 64 keys]  = Q [128 x D] . K^T            (tcgen05.mma, S in tensor memory)
+//     O [128 rows x D]       += P [128 x 64 keys] . V        (P bf16 in shared memory, O in tensor memory)
+//
+// Warp roles (192 threads):
+//   warp 4, one lane -- producer: loads each unit's Q tile (one TMA box of G
+//     heads x max_q tokens, right-aligned so it ends at the sequence's last
+//     query token; rows past the sequence's own tokens are never written)
+//     into one of two Q buffers, then streams the unit's K and V tiles into a
+//     ring of shared-memory stages exactly like the warp-MMA kernel;
+//   warp 5, one lane -- MMA issuer: S(j) = Q K_j^T into one of two S buffers,
+//     then O += P(j-1) V_{j-1}, so the softmax of tile j overlaps the second
+//     product of tile j-1 (a unit's last tile is not held back: its second
+//     product follows at once); completion is tracked with tcgen05.commit on
+//     mbarriers; the warp also allocates and frees the tensor memory;
+//   warps 0-3 -- softmax and epilogue, thread r owning query row r (tensor
+//     memory lane r): it reads its 64 scores of S(j), masks them (the keys
+//     before the tile's own start when the tile was right-aligned, and under
+//     the tail-aligned causal mask, keys past Lk - Lq + qi), runs the online
+//     softmax in base-2 units and writes its row of P(j) as bf16 into the
+//     128-byte swizzled operand layout.
+//
+// The running max is rescaled lazily: O in tensor memory is multiplied by
+// 2^(m_old - m_new) only when a row's max grows by more than 2^8 (rare after
+// the first tile); otherwise the tile's weights are taken relative to the
+// stale max, which stays exact in fp32 and keeps P below 2^8 in bf16.  The
+// partial (O, m, l) and the final normalisation use whatever reference max
+// the row ended with, so the result is the same softmax.
+//
+// Every wait on an mbarrier is bounded; a wait that gives up records
+// ATTN_DEV_ERR_TIMEOUT, raises a block-wide stop flag that the other roles'
+// waits also watch, and the block drains its issued tensor-core work before
+// freeing the tensor memory and returning.
+#include "common.cuh"
+#include "kernels.h"
+#include "schedule.cuh"
+#include "tc.cuh"
+
+namespace vgqa {
+
+namespace {
+
+using namespace sched;
+
+constexpr int kRows = 128;                // MMA M: query rows of a unit
+constexpr int kSoftWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kThreads = 192;
+constexpr int kMetaLast = 1;              // stage flag: the block's last tile of the unit
+constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends here
+constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold (base-2 units)
+constexpr uint32_t kTmemCols = 256;       // S buffers at columns [0, 128), O at [128, 128 + D)
+constexpr uint32_t kColS = 0, kColO = 128;
+
+template <int D>
+struct TcLayout {
+    static constexpr int kHalves = D / 64;                  // 128-byte swizzle atoms per row
+    static constexpr int kKvRegion = kBN * 128;             // 64 keys x 128 B
+    static constexpr int kKvTile = kHalves * kKvRegion;     // K or V tile
+    static constexpr int kStage = 2 * kKvTile;              // K + V
+    static constexpr int kQRegion = kRows * 128;            // 128 rows x 128 B
+    static constexpr int kQTile = kHalves * kQRegion;
+    static constexpr int kPTile = kRows * 128;              // 128 rows x 64 keys bf16
+};
+
+// bounded mbarrier wait that also gives up when another role raised the stop flag
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *stop, const Params &p) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*stop) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
+            *stop = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                               const __grid_constant__ CUtensorMap tm_k,
+                                                               const __grid_constant__ CUtensorMap tm_v,
+                                                               const Params p, const int stages) {
+    using L = TcLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ring = smem;                                    // [stages][K tile | V tile]
+    uint8_t *qbuf = ring + stages * L::kStage;               // [2][Q tile]
+    uint8_t *pbuf = qbuf + 2 * L::kQTile;                    // P tile
+    uint64_t *full = reinterpret_cast<uint64_t *>(pbuf + L::kPTile);
+    uint64_t *empty = full + stages;
+    uint64_t *q_full = empty + stages;       // [2] Q tile landed
+    uint64_t *q_free = q_full + 2;           // [2] last product reading the Q tile done
+    uint64_t *s_full = q_free + 2;           // [2] S(j) computed
+    uint64_t *s_free = s_full + 2;           // [2] S(j) read by the softmax warps
+    uint64_t *p_full = s_free + 2;           // P(j) written
+    uint64_t *o_done = p_full + 1;           // [2] O += P(j) V(j) done (j mod 2)
+    uint64_t *o_free = o_done + 2;           // O read by the epilogue
+    uint64_t *drain = o_free + 1;            // all issued tensor-core work done
+    int2 *meta = reinterpret_cast<int2 *>(drain + 1);                         // [stages]
+    long long *scan = reinterpret_cast<long long *>(meta + stages);          // [8]
+    long long *first = scan + 8;                                             // [3]
+    volatile int *stop = reinterpret_cast<volatile int *>(first + 3);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(first + 3) + 1;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x;
+
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + kSoftWarps);   // the MMA's commit (or arrival) + each softmax warp
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_free[i], 1);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], kSoftWarps);
+            mbar_init(&o_done[i], 1);
+        }
+        mbar_init(p_full, kSoftWarps);
+        mbar_init(o_free, kSoftWarps);
+        mbar_init(drain, 1);
+        *stop = 0;
+        fence_barrier_init();
+    }
+    if (tid == kProducerWarp * 32) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    if (warp == kMmaWarp) {
+        tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    // Launched as a programmatic dependent, the block may start while the
+    // previous kernel in the stream still runs; everything above touches only
+    // this block's shared and tensor memory.  Wait for that kernel before
+    // reading global memory; only then may this call's combine kernel launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    Share sh;
+    const bool has_work = block_share(p, c, gridDim.x, tid, kThreads, c == 0, scan, first, sh);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const int G = p.G, QT = p.max_q;
+
+    if (has_work && warp == kProducerWarp && lane == 0) {
+        // ---------------------------------------------------------- producer
+        const uint64_t pol = l2_evict_first();
+        const uint32_t q_bytes = (uint32_t)(L::kHalves * G * QT * 128);
+        int s = 0, issued = 0, k = 0;
+        uint32_t phase = 0;
+        auto acquire = [&]() -> bool { return issued < stages || wait_bar(&empty[s], phase ^ 1, stop, p); };
+        auto advance = [&]() {
+            ++issued;
+            if (++s == stages) {
+                s = 0;
+                phase ^= 1;
+            }
+        };
+        auto begin = [&](const Segment &sg, int) -> bool {
+            const int qb = k & 1;
+            if (k >= 2 && !wait_bar(&q_free[qb], ((k - 2) >> 1) & 1, stop, p)) return false;
+            mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+            const int t_end = sg.s.q0 + sg.s.Lq;             // box ends at the sequence's last query token
+#pragma unroll
+            for (int hf = 0; hf < L::kHalves; ++hf)
+                tma_load_3d(qbuf + qb * L::kQTile + hf * L::kQRegion, &tm_q, &q_full[qb], hf * 64, sg.hk * G,
+                            t_end - QT, pol);
+            ++k;
+            return true;
+        };
+        auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
+            if (!acquire()) return false;
+            const int ks = tile * kBN;
+            const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
+            meta[s] = make_int2(ks, last ? kMetaLast : 0);
+            uint8_t *st = ring + s * L::kStage;
+            mbar_arrive_expect_tx(&full[s], L::kStage);
+#pragma unroll
+            for (int hf = 0; hf < L::kHalves; ++hf)
+                tma_load_3d(st + hf * L::kKvRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
+#pragma unroll
+            for (int hf = 0; hf < L::kHalves; ++hf)
+                tma_load_3d(st + L::kKvTile + hf * L::kKvRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
+            advance();
+            return true;
+        };
+        auto empty_stage = [&](const Segment &) -> bool {
+            if (!acquire()) return false;
+            meta[s] = make_int2(0, kMetaLast | kMetaEmpty);
+            mbar_arrive(&full[s]);
+            advance();
+            return true;
+        };
+        if (!feed_tiles(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage)) *stop = 1;
+        // let the loads in flight land before the block can exit (bounded,
+        // also after a stop: the copies target this block's shared memory)
+        for (int i = 0; i < min(issued, stages); ++i) {
+            if (--s < 0) {
+                s = stages - 1;
+                phase ^= 1;
+            }
+            mbar_wait(&full[s], phase);
+        }
+        if (k >= 1) mbar_wait(&q_full[(k - 1) & 1], ((k - 1) >> 1) & 1);
+        if (k >= 2) mbar_wait(&q_full[k & 1], ((k - 2) >> 1) & 1);
+    } else if (has_work && warp == kMmaWarp) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdS = tc::idesc_bf16_f32(kRows, kBN, false);
+            constexpr uint32_t kIdO = tc::idesc_bf16_f32(kRows, D, true);
+            const uint32_t ring0 = smem_u32(ring), q0 = smem_u32(qbuf), p0 = smem_u32(pbuf);
+            int j = 0, st = 0, k = 0, e = 0;
+            bool have_prev = false, ok = true;
+            int pj = 0, ps = 0, pe = 0;
+            bool pfirst = false;
+            // O += P(pj) V(pj): waits for the softmax warps' P and, at a
+            // unit's first tile, for the epilogue of the previous unit
+            auto issue_pv = [&]() -> bool {
+                if (!wait_bar(p_full, pj & 1, stop, p)) return false;
+                if (pfirst && pe >= 1 && !wait_bar(o_free, (pe - 1) & 1, stop, p)) return false;
+                tc::fence_after_sync();
+                const uint32_t v0 = ring0 + ps * L::kStage + L::kKvTile;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    const uint64_t a = tc::smem_desc_sw128(p0 + kk * 32, 16, 1024);
+                    const uint64_t b = tc::smem_desc_sw128(v0 + kk * 16 * 128, L::kKvRegion, 1024);
+                    tc::mma_bf16_ss(tmem + kColO, a, b, kIdO, !pfirst || kk > 0);
+                }
+                tc::commit(smem_u32(&empty[ps]));
+                tc::commit(smem_u32(&o_done[pj & 1]));
+                return true;
+            };
+            OrderedWalker wk;
+            wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
+            Segment seg;
+            int role;
+            while (ok && wk.next(p, seg, role)) {
+                const int qb = k & 1;
+                if (!(ok = wait_bar(&q_full[qb], (k >> 1) & 1, stop, p))) break;
+                const uint32_t qa = q0 + qb * L::kQTile;
+                bool first = true;
+                while (true) {
+                    const int s = st % stages;
+                    if (!(ok = wait_bar(&full[s], (st / stages) & 1, stop, p))) break;
+                    const int2 mt = meta[s];
+                    ++st;
+                    if (mt.y & kMetaEmpty) {            // the unit ends without a tile here
+                        mbar_arrive(&empty[s]);
+                        mbar_arrive(&q_free[qb]);
+                        break;
+                    }
+                    const int b = j & 1;
+                    if (j >= 2 && !(ok = wait_bar(&s_free[b], ((j - 2) >> 1) & 1, stop, p))) break;
+                    tc::fence_after_sync();
+                    const uint32_t k0 = ring0 + s * L::kStage;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int hf = kk >> 2, cc = (kk & 3) * 32;
+                        const uint64_t a = tc::smem_desc_sw128(qa + hf * L::kQRegion + cc, 16, 1024);
+                        const uint64_t bd = tc::smem_desc_sw128(k0 + hf * L::kKvRegion + cc, 16, 1024);
+                        tc::mma_bf16_ss(tmem + kColS + b * kBN, a, bd, kIdS, kk > 0);
+                    }
+                    tc::commit(smem_u32(&s_full[b]));
+                    if (mt.y & kMetaLast) tc::commit(smem_u32(&q_free[qb]));
+                    if (have_prev && !(ok = issue_pv())) break;
+                    have_prev = true;
+                    pj = j;
+                    ps = s;
+                    pfirst = first;
+                    pe = e;
+                    first = false;
+                    ++j;
+                    if (mt.y & kMetaLast) {
+                        // the unit's last product goes out now: the epilogue
+                        // waits for it, and the next tile may be several
+                        // (empty) units away
+                        if (!(ok = issue_pv())) break;
+                        have_prev = false;
+                        ++e;
+                        break;
+                    }
+                }
+                ++k;
+            }
+            if (ok && have_prev) ok = issue_pv();
+            if (!ok) *stop = 1;
+            // nothing this thread issued may still run when the memory is freed
+            tc::commit(smem_u32(drain));
+            mbar_wait(drain, 0);
+        }
+        __syncwarp();
+    } else if (has_work && warp < kSoftWarps) {
+        // ---------------------------------------------------------- softmax + epilogue
+        const int r = tid;                                   // query row = tensor-memory lane
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float cs = p.scale_log2;
+        uint8_t *prow = pbuf + r * 128;
+        // every lane waits; the warp goes on only if all of them succeeded,
+        // so the warp-collective tensor-memory accesses stay converged
+        auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            const bool w = wait_bar(bar, parity, stop, p);
+            return __all_sync(0xffffffffu, w);
+        };
+        int j = 0, st = 0;
+        bool ok = true;
+        OrderedWalker wk;
+        wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
+        Segment seg;
+        int role;
+        while (ok && wk.next(p, seg, role)) {
+            const int Lq = seg.s.Lq, Lk = seg.s.Lk;
+            const int tq = r / G, g = r - tq * G;
+            const int qi = tq - (QT - Lq);                       // this row's query token in the sequence
+            const bool valid = tq < QT && qi >= 0;
+            const int vis = valid ? Lk - Lq + qi + 1 : 0;        // keys [0, vis) visible (tail-aligned causal)
+            float m_used = -INFINITY, l = 0.f;
+            bool first = true, has_tiles = false;
+            while (true) {
+                const int s = st % stages;
+                if (!(ok = wwait(&full[s], (st / stages) & 1))) break;
+                const int2 mt = meta[s];
+                ++st;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (mt.y & kMetaEmpty) break;
+                has_tiles = true;
+                const int b = j & 1;
+                if (!(ok = wwait(&s_full[b], (j >> 1) & 1))) break;
+                tc::fence_after_sync();
+                uint32_t sa[32], sb[32];
+                tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kBN, sa);
+                tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kBN + 32, sb);
+                tc::wait_ld();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[b]);
+
+                // mask and tile max, in base-2 units of the scaled scores
+                const int ks = mt.x, ls = min(ks, Lk - kBN);     // key of column 0
+                const int lo_c = ks - ls, hi_c = min(kBN, vis - ls);   // visible columns [lo_c, hi_c)
+                float x[kBN];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int cc = 0; cc < 32; ++cc) {
+                    x[cc] = (cc >= lo_c && cc < hi_c) ? __uint_as_float(sa[cc]) * cs : -INFINITY;
+                    x[cc + 32] = (cc + 32 >= lo_c && cc + 32 < hi_c) ? __uint_as_float(sb[cc]) * cs : -INFINITY;
+                    mx = fmaxf(mx, fmaxf(x[cc], x[cc + 32]));
+                }
+                const bool need = mx > m_used + kRescaleLog2;    // false while the tile has no visible key
+                const float m_new = need ? mx : m_used;
+                bool o_ready = false;                            // O += P(j-1) V(j-1) known done
+                if (!first && __any_sync(0xffffffffu, need)) {
+                    if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
+                    o_ready = true;
+                    tc::fence_after_sync();
+                    const float alpha = need ? ex2(m_used - m_new) : 1.f;
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t o[32];
+                        tc::ld_32x32b_x32(tmem + lane_base + kColO + ch * 32, o);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tc::st_32x32b_x32(tmem + lane_base + kColO + ch * 32, o);
+                    }
+                    tc::wait_st();
+                }
+                if (need) {
+                    l *= ex2(m_used - m_new);                     // ex2(-inf) = 0 on the first visible key
+                    m_used = m_new;
+                }
+                const float mref = m_used == -INFINITY ? 0.f : m_used;
+                uint32_t pk[kBN / 2];
+                float lt = 0.f;
+#pragma unroll
+                for (int i = 0; i < kBN / 2; ++i) {
+                    const float p0 = ex2(x[2 * i] - mref), p1 = ex2(x[2 * i + 1] - mref);
+                    lt += p0 + p1;
+                    pk[i] = pack_bf16x2(p0, p1);
+                }
+                l += lt;
+                // the single P buffer is free once O += P(j-1) V(j-1) is done
+                if (j >= 1 && !o_ready && !(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1)))
+                    break;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                    *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = v4;
+                }
+                fence_proxy_async();                             // generic writes -> tensor-core reads
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full);
+                first = false;
+                ++j;
+                if (mt.y & kMetaLast) break;
+            }
+            if (!ok) break;
+
+            // ---------------- epilogue: this block's part of the unit
+            if (has_tiles) {
+                if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
+                tc::fence_after_sync();
+            }
+            const bool whole = role == 0;
+            const int slot = role == 1 ? 2 * c : 2 * c + 1;
+            const int pr = qi * G + g;                            // row within the unit's G * Lq rows
+            const long long tok = seg.s.q0 + qi;
+            const int h = seg.hk * G + g;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            if (has_tiles) {
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t o[32];
+                    __syncwarp();
+                    tc::ld_32x32b_x32(tmem + lane_base + kColO + ch * 32, o);   // warp-collective
+                    tc::wait_ld();
+                    if (!valid) {
+                    } else if (whole) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D + ch * 32);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+                            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+                            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+                            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+                            dst[v] = w;
+                        }
+                    } else {
+                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((long long)slot * kRows + pr) * D + ch * 32);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                    }
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(o_free);
+            } else if (valid && whole) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D);
+#pragma unroll
+                for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (valid) {
+                if (whole)
+                    p.lse[tok * p.Hq + h] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+                else
+                    p.ml_part[(long long)slot * kRows + pr] = make_float2(m_used, l);
+            }
+            // publish this warp's rows of the part (the combine waits for all
+            // kSoftWarps warps of each of the unit's n blocks)
+            if (!whole) {
+                __syncwarp();
+                if (lane == 0) red_add_release_gpu(p.done + (long long)seg.b * p.Hkv + seg.hk, 1u);
+            }
+        }
+        if (!ok) *stop = 1;
+    }
+
+    // free the tensor memory once every role is done with it
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D>
+void *tc_kernel_ptr() {
+    return reinterpret_cast<void *>(split_tc_kernel<D>);
+}
+
+}  // namespace
+
+size_t tc_stage_bytes(int D) { return D == 64 ? TcLayout<64>::kStage : TcLayout<128>::kStage; }
+
+size_t tc_smem_bytes(int D, int stages) {
+    const size_t fixed = D == 64 ? 2 * TcLayout<64>::kQTile + TcLayout<64>::kPTile
+                                 : 2 * TcLayout<128>::kQTile + TcLayout<128>::kPTile;
+    // 1 KB alignment slack + ring + Q tiles + P tile + barriers + meta + scan + (first, T) + stop flag, tmem slot
+    return 1024 + tc_stage_bytes(D) * stages + fixed + (2 * stages + 14) * 8 + stages * 8 + (8 + 3) * 8 + 16;
+}
+
+int tc_rows() { return kRows; }
+int tc_parts_per_block() { return kSoftWarps; }
+
+cudaError_t tc_prepare(int D, int stages, int ctas) {
+    void *fn = D == 64 ? tc_kernel_ptr<64>() : tc_kernel_ptr<128>();
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(D, stages));
+    if (e != cudaSuccess) return e;
+    return combine_slots_prepare(D, ctas);
+}
+
+cudaError_t launch_split_tc(const Params &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                            const CUtensorMap &tm_v, int stages, int ctas, cudaStream_t stream) {
+    // programmatic dependent launches, as for the warp-MMA kernel
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = tc_smem_bytes(p.D, stages);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int st = stages;
+    void *args[] = {const_cast<CUtensorMap *>(&tm_q), const_cast<CUtensorMap *>(&tm_k),
+                    const_cast<CUtensorMap *>(&tm_v), const_cast<Params *>(&p), &st};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, p.D == 64 ? tc_kernel_ptr<64>() : tc_kernel_ptr<128>(), args);
+    if (e != cudaSuccess) return e;
+    return launch_combine_slots(p, ctas, stream);
+}
+
+}  // namespace vgqa
