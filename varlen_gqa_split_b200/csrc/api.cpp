@@ -194,7 +194,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         d.grid_z = 1;
         d.deterministic = o && o->deterministic ? 1 : 0;
         d.combine = ATTN_COMBINE_KERNEL;     // slot-parallel combine, programmatic dependent launch
-        d.combine_blocks = 2 * d.ctas;
+        d.combine_blocks = 2 * d.ctas * combine_slots_split((int)rows, D);
         n_ticket = 3 * (size_t)B_max * Hkv;  // per cut unit: tile claims (64-bit), part count
         n_part = 2 * (size_t)d.ctas;       // two partial slots per block
         part_rows = d.rows_per_block;

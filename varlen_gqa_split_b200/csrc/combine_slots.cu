@@ -33,19 +33,22 @@ using namespace sched;
 // while the split kernel streams; it then waits (bounded) only for the n parts
 // of its own unit, whose writers each add 1 (release) to the unit's count, so
 // a unit is merged as soon as its last part lands rather than when the whole
-// split grid ends.  After merging, each of the unit's n combine blocks adds 1
-// again; the one that brings the count to 2n resets it for the next call.
+// split grid ends.  Each slot's slice is cut again into S sub-slices, one per
+// block, so that a unit with many rows is merged by n * S blocks.  After
+// merging, each of the unit's n * S combine blocks adds 1 to the count again;
+// the last one resets it for the next call.
 template <int D>
-__global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, const int C) {
+__global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, const int C, const int S) {
     constexpr int kCols = D / 4;
     constexpr int kT = 128;
     constexpr int kBatch = 12;             // loads in flight per thread (register budget)
     extern __shared__ __align__(16) uint8_t csm[];
-    __shared__ long long scan[8];
+    __shared__ long long scan[kT / 32];
     __shared__ long long first[3];
     __shared__ int ok_flag;
     const int tid = threadIdx.x;
-    const int c = blockIdx.x >> 1, k = blockIdx.x & 1;
+    const int sub = blockIdx.x % S;
+    const int c = (blockIdx.x / S) >> 1, k = (blockIdx.x / S) & 1;
     const long long ROWS = p.rows_per_block;     // rows of one partial slot
     // the next call's split kernel may launch now; it waits for this grid to
     // complete before it reads anything
@@ -69,8 +72,9 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
     const int n = block_of(seg.Pu + seg.s.tpu - 1, T, Ce) - c_first + 1;
     const int G = p.G, R = G * seg.s.Lq;
     const int items = R * kCols;
-    const int per = (items + n - 1) / n;
-    const int it_lo = min(items, (c - c_first) * per), it_hi = min(items, it_lo + per);
+    const int nb = n * S;                          // blocks merging this unit
+    const int per = (items + nb - 1) / nb;
+    const int it_lo = min(items, ((c - c_first) * S + sub) * per), it_hi = min(items, it_lo + per);
     const long long u = (long long)seg.b * p.Hkv + seg.hk;
 
     int *slots = reinterpret_cast<int *>(csm);                         // [n]
@@ -93,7 +97,7 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
             }
         }
         ok_flag = ok;
-        if (ok && c == c_first) p.claim[u] = 0ull;                      // claims, next call
+        if (ok && c == c_first && sub == 0) p.claim[u] = 0ull;          // claims, next call
     }
     __syncthreads();
     if (!ok_flag) return;
@@ -161,8 +165,8 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
     }
     __syncthreads();
     // every combine block of the unit has seen its n parts once each of the
-    // n blocks has added 1 more: the last one resets the count
-    if (tid == 0 && atomicAdd(p.done + u, 1u) == parts_done + (uint32_t)(n - 1)) p.done[u] = 0u;
+    // n * S blocks has added 1 more: the last one resets the count
+    if (tid == 0 && atomicAdd(p.done + u, 1u) == parts_done + (uint32_t)(nb - 1)) p.done[u] = 0u;
 }
 
 
@@ -177,6 +181,13 @@ cudaError_t combine_slots_prepare(int D, int ctas) {
     return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)combine_slots_smem(ctas));
 }
 
+int combine_slots_split(int rows, int D) {
+    // about 512 (row, 4-column) items per block at most, up to 8 blocks per slot
+    const int items = rows * (D / 4);
+    const int S = (items + 511) / 512;
+    return S < 1 ? 1 : (S > 8 ? 8 : S);
+}
+
 cudaError_t launch_combine_slots(const Params &p, int ctas, cudaStream_t stream) {
     // launched as a programmatic dependent: its blocks may start (and compute
     // the schedule) before the split kernel has finished
@@ -184,7 +195,8 @@ cudaError_t launch_combine_slots(const Params &p, int ctas, cudaStream_t stream)
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(2 * ctas);
+    int S = combine_slots_split(p.G * p.max_q, p.D);
+    cfg.gridDim = dim3(2 * ctas * S);
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = combine_slots_smem(ctas);
     cfg.stream = stream;
@@ -192,7 +204,7 @@ cudaError_t launch_combine_slots(const Params &p, int ctas, cudaStream_t stream)
     cfg.numAttrs = 1;
     void *fn = p.D == 64 ? reinterpret_cast<void *>(combine_slots_kernel<64>)
                          : reinterpret_cast<void *>(combine_slots_kernel<128>);
-    void *args[] = {const_cast<Params *>(&p), &ctas};
+    void *args[] = {const_cast<Params *>(&p), &ctas, &S};
     return cudaLaunchKernelExC(&cfg, fn, args);
 }
 

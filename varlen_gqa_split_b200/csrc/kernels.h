@@ -41,6 +41,7 @@ cudaError_t launch_split_tc(const Params &p, const CUtensorMap &tm_q, const CUte
 // log-sum-exp merge of the persistent kernels' partial slots (2 * ctas
 // blocks, launched as a programmatic dependent of the split kernel)
 size_t combine_slots_smem(int ctas);
+int combine_slots_split(int rows, int D);   // blocks per partial slot (S)
 cudaError_t combine_slots_prepare(int D, int ctas);
 cudaError_t launch_combine_slots(const Params &p, int ctas, cudaStream_t stream);
 

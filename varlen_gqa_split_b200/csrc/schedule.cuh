@@ -178,14 +178,14 @@ __device__ __forceinline__ int slot_of(int c, long long Pu, long long T, int C) 
 // threads of the block from cu_seqlens.  Each thread weighs a contiguous run of
 // sequences; a scan of the run totals gives the tile prefix, the total T and
 // the share; the thread whose run holds the share's first tile finds its unit.
-// scan: 8 long long, first: 3 long long of shared memory.
 struct Share {
     long long T, lo, hi, pb_first;
     int Ce, b_first;
 };
 
+// scan: nthreads / 32 long long of shared memory (one per warp); first: 3.
 __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int tid, int nthreads, bool report,
-                            long long *scan, long long *first, Share &sh) {
+                                            long long *scan, long long *first, Share &sh) {
     const int warp = tid >> 5, lane = tid & 31;
     const int per = (p.B_max + nthreads - 1) / nthreads;
     const int b_lo = min(p.B_max, tid * per), b_hi = min(p.B_max, b_lo + per);

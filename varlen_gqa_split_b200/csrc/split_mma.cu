@@ -43,6 +43,7 @@ using namespace sched;
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
+static_assert(kThreads / 32 <= 8, "block_share scan scratch holds 8 warps");
 constexpr int kBarConsumers = 1;          // named barrier of the consumer warps
 constexpr int kMetaLast = 1;              // stage flag: the block's last tile of the unit
 constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends here
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     uint64_t *empty = full + stages;
     int2 *meta = reinterpret_cast<int2 *>(empty + stages);                       // [stages] (key start, flags)
     long long *scan = reinterpret_cast<long long *>(meta + stages + (stages & 1)); // [warps]
-    long long *first = scan + 8;                                                 // b_first, pb_first, T
+    long long *first = scan + 8;                         // b_first, pb_first, T (scan: kThreads / 32 <= 8)
     volatile int *flags = reinterpret_cast<volatile int *>(first + 3);          // failed
 
     const int tid = threadIdx.x;

@@ -11,25 +11,30 @@
 //     S [128 rows x 64 keys]  = Q [128 x D] . K^T            (tcgen05.mma, S in tensor memory)
 //     O [128 rows x D]       += P [128 x 64 keys] . V        (P bf16 in shared memory, O in tensor memory)
 //
-// Warp roles (192 threads):
-//   warp 4, one lane -- producer: loads each unit's Q tile (one TMA box of G
+// Warp roles (320 threads):
+//   warp 8, one lane -- producer: loads each unit's Q tile (one TMA box of G
 //     heads x max_q tokens, right-aligned so it ends at the sequence's last
 //     query token; rows past the sequence's own tokens are never written)
 //     into one of two Q buffers, then streams the unit's K and V tiles into a
 //     ring of shared-memory stages exactly like the warp-MMA kernel;
-//   warp 5, one lane -- MMA issuer: S(j) = Q K_j^T into one of two S buffers,
+//   warp 9, one lane -- MMA issuer: S(j) = Q K_j^T into one of two S buffers,
 //     then O += P(j-1) V_{j-1}, so the softmax of tile j overlaps the second
 //     product of tile j-1 (a unit's last tile is not held back: its second
 //     product follows at once); completion is tracked with tcgen05.commit on
 //     mbarriers; the warp also allocates and frees the tensor memory;
-//   warps 0-3 -- softmax and epilogue, thread r owning query row r (tensor
-//     memory lane r): it reads its 64 scores of S(j), masks them (the keys
-//     before the tile's own start when the tile was right-aligned, and under
-//     the tail-aligned causal mask, keys past Lk - Lq + qi), runs the online
-//     softmax in base-2 units and writes its row of P(j) as bf16 into the
+//   warps 0-7 -- softmax and epilogue.  Warp w reads tensor-memory lanes
+//     32 (w mod 4) .. +31, one query row per thread, and column half
+//     h = w / 4 of every tile (keys 32h .. 32h+31).  Each half runs its own
+//     online softmax in base-2 units over its keys and accumulates its own
+//     O_h (the product P[:, half h] V[half h] goes to a separate tensor-memory
+//     accumulator), so the two warps of a row never synchronise per tile;
+//     the epilogue merges the two halves like two split-KV partials.  The
+//     scores are masked (keys before the tile's own start when the tile was
+//     right-aligned, and keys past Lk - Lq + qi under the tail-aligned causal
+//     mask), and P is written as bf16 into one of two P buffers in the
 //     128-byte swizzled operand layout.
 //
-// The running max is rescaled lazily: O in tensor memory is multiplied by
+// The running max is rescaled lazily: O_h in tensor memory is multiplied by
 // 2^(m_old - m_new) only when a row's max grows by more than 2^8 (rare after
 // the first tile); otherwise the tile's weights are taken relative to the
 // stale max, which stays exact in fp32 and keeps P below 2^8 in bf16.  The
@@ -52,15 +57,18 @@ namespace {
 using namespace sched;
 
 constexpr int kRows = 128;                // MMA M: query rows of a unit
-constexpr int kSoftWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;             // two per tensor-memory lane quarter (column halves)
+constexpr int kEpiWarps = 4;              // the half-0 warps write the outputs
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr int kHalfKeys = kBN / 2;
 constexpr int kMetaLast = 1;              // stage flag: the block's last tile of the unit
 constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends here
 constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold (base-2 units)
-constexpr uint32_t kTmemCols = 256;       // S buffers at columns [0, 128), O at [128, 128 + D)
-constexpr uint32_t kColS = 0, kColO = 128;
+constexpr uint32_t kTmemCols = 512;       // S buffers [0, 128), O_0 [128, 128 + D), O_1 [256, 256 + D)
+constexpr uint32_t kColS = 0, kColO0 = 128, kColO1 = 256;
+constexpr size_t kMinSmemBytes = 120 * 1024;
 
 template <int D>
 struct TcLayout {
@@ -98,20 +106,22 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;                                    // [stages][K tile | V tile]
     uint8_t *qbuf = ring + stages * L::kStage;               // [2][Q tile]
-    uint8_t *pbuf = qbuf + 2 * L::kQTile;                    // P tile
-    uint64_t *full = reinterpret_cast<uint64_t *>(pbuf + L::kPTile);
+    uint8_t *pbuf = qbuf + 2 * L::kQTile;                    // [2][P tile]
+    uint64_t *full = reinterpret_cast<uint64_t *>(pbuf + 2 * L::kPTile);
     uint64_t *empty = full + stages;
     uint64_t *q_full = empty + stages;       // [2] Q tile landed
     uint64_t *q_free = q_full + 2;           // [2] last product reading the Q tile done
-    uint64_t *s_full = q_free + 2;           // [2] S(j) computed
+    uint64_t *s_full = q_free + 2;           // [2] S(j) computed (j mod 2)
     uint64_t *s_free = s_full + 2;           // [2] S(j) read by the softmax warps
-    uint64_t *p_full = s_free + 2;           // P(j) written
-    uint64_t *o_done = p_full + 1;           // [2] O += P(j) V(j) done (j mod 2)
-    uint64_t *o_free = o_done + 2;           // O read by the epilogue
-    uint64_t *drain = o_free + 1;            // all issued tensor-core work done
+    uint64_t *p_full = s_free + 2;           // [2] P(j) written
+    uint64_t *o_done = p_full + 2;           // [2] O += P(j) V(j) done
+    uint64_t *o_free = o_done + 2;           // O_0, O_1 read by the epilogue
+    uint64_t *xch = o_free + 1;              // half-1 (m, l) of a unit published
+    uint64_t *drain = xch + 1;               // all issued tensor-core work done
     int2 *meta = reinterpret_cast<int2 *>(drain + 1);                         // [stages]
-    long long *scan = reinterpret_cast<long long *>(meta + stages);          // [8]
-    long long *first = scan + 8;                                             // [3]
+    float2 *xml = reinterpret_cast<float2 *>(meta + stages);                 // [128] half-1 (m, l)
+    long long *scan = reinterpret_cast<long long *>(xml + kRows);            // [kThreads / 32]
+    long long *first = scan + kThreads / 32;                                 // [3]
     volatile int *stop = reinterpret_cast<volatile int *>(first + 3);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(first + 3) + 1;
 
@@ -129,10 +139,11 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             mbar_init(&q_free[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&s_free[i], kSoftWarps);
+            mbar_init(&p_full[i], kSoftWarps);
             mbar_init(&o_done[i], 1);
         }
-        mbar_init(p_full, kSoftWarps);
-        mbar_init(o_free, kSoftWarps);
+        mbar_init(o_free, kEpiWarps);
+        mbar_init(xch, kSoftWarps - kEpiWarps);
         mbar_init(drain, 1);
         *stop = 0;
         fence_barrier_init();
@@ -232,19 +243,24 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             bool have_prev = false, ok = true;
             int pj = 0, ps = 0, pe = 0;
             bool pfirst = false;
-            // O += P(pj) V(pj): waits for the softmax warps' P and, at a
-            // unit's first tile, for the epilogue of the previous unit
+            // O_h += P(pj)[:, half h] V(pj)[half h]: waits for the softmax
+            // warps' P and, at a unit's first tile, for the epilogue of the
+            // previous unit
             auto issue_pv = [&]() -> bool {
-                if (!wait_bar(p_full, pj & 1, stop, p)) return false;
+                if (!wait_bar(&p_full[pj & 1], (pj >> 1) & 1, stop, p)) return false;
                 if (pfirst && pe >= 1 && !wait_bar(o_free, (pe - 1) & 1, stop, p)) return false;
                 tc::fence_after_sync();
                 const uint32_t v0 = ring0 + ps * L::kStage + L::kKvTile;
+                const uint32_t pa = p0 + (pj & 1) * L::kPTile;
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint64_t a = tc::smem_desc_sw128(p0 + kk * 32, 16, 1024);
-                    const uint64_t b = tc::smem_desc_sw128(v0 + kk * 16 * 128, L::kKvRegion, 1024);
-                    tc::mma_bf16_ss(tmem + kColO, a, b, kIdO, !pfirst || kk > 0);
-                }
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < kHalfKeys / 16; ++kk) {
+                        const int key = h * kHalfKeys + kk * 16;
+                        const uint64_t a = tc::smem_desc_sw128(pa + key * 2, 16, 1024);
+                        const uint64_t b = tc::smem_desc_sw128(v0 + key * 128, L::kKvRegion, 1024);
+                        tc::mma_bf16_ss(tmem + (h ? kColO1 : kColO0), a, b, kIdO, !pfirst || kk > 0);
+                    }
                 tc::commit(smem_u32(&empty[ps]));
                 tc::commit(smem_u32(&o_done[pj & 1]));
                 return true;
@@ -310,17 +326,18 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         __syncwarp();
     } else if (has_work && warp < kSoftWarps) {
         // ---------------------------------------------------------- softmax + epilogue
-        const int r = tid;                                   // query row = tensor-memory lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = quarter * 32 + lane;                   // query row = tensor-memory lane
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t col_o = half ? kColO1 : kColO0;
         const float cs = p.scale_log2;
-        uint8_t *prow = pbuf + r * 128;
         // every lane waits; the warp goes on only if all of them succeeded,
         // so the warp-collective tensor-memory accesses stay converged
         auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
             const bool w = wait_bar(bar, parity, stop, p);
             return __all_sync(0xffffffffu, w);
         };
-        int j = 0, st = 0;
+        int j = 0, st = 0, e = 0;
         bool ok = true;
         OrderedWalker wk;
         wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
@@ -346,41 +363,47 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 const int b = j & 1;
                 if (!(ok = wwait(&s_full[b], (j >> 1) & 1))) break;
                 tc::fence_after_sync();
-                uint32_t sa[32], sb[32];
-                tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kBN, sa);
-                tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kBN + 32, sb);
+                uint32_t sv[kHalfKeys];
+                tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kBN + half * kHalfKeys, sv);
                 tc::wait_ld();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_free[b]);
 
-                // mask and tile max, in base-2 units of the scaled scores
+                // mask and max of this half.  The scale (> 0) enters in the
+                // exp2 argument, so the raw maximum gives the scaled one; a
+                // masked score becomes -inf, whose weight is exactly 0.
                 const int ks = mt.x, ls = min(ks, Lk - kBN);     // key of column 0
-                const int lo_c = ks - ls, hi_c = min(kBN, vis - ls);   // visible columns [lo_c, hi_c)
-                float x[kBN];
-                float mx = -INFINITY;
+                const int c0 = half * kHalfKeys;
+                const int lo_c = ks - ls - c0, hi_c = min(kHalfKeys, vis - ls - c0);   // visible [lo_c, hi_c)
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (__all_sync(0xffffffffu, lo_c <= 0 && hi_c >= kHalfKeys)) {
 #pragma unroll
-                for (int cc = 0; cc < 32; ++cc) {
-                    x[cc] = (cc >= lo_c && cc < hi_c) ? __uint_as_float(sa[cc]) * cs : -INFINITY;
-                    x[cc + 32] = (cc + 32 >= lo_c && cc + 32 < hi_c) ? __uint_as_float(sb[cc]) * cs : -INFINITY;
-                    mx = fmaxf(mx, fmaxf(x[cc], x[cc + 32]));
+                    for (int cc = 0; cc < kHalfKeys; ++cc) mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(sv[cc]));
+                } else {
+#pragma unroll
+                    for (int cc = 0; cc < kHalfKeys; ++cc) {
+                        if (cc < lo_c || cc >= hi_c) sv[cc] = 0xff800000u;   // -inf
+                        mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(sv[cc]));
+                    }
                 }
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * cs;
                 const bool need = mx > m_used + kRescaleLog2;    // false while the tile has no visible key
                 const float m_new = need ? mx : m_used;
-                bool o_ready = false;                            // O += P(j-1) V(j-1) known done
                 if (!first && __any_sync(0xffffffffu, need)) {
+                    // O_h holds P V of earlier tiles: rescale it once their
+                    // products are done
                     if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
-                    o_ready = true;
                     tc::fence_after_sync();
                     const float alpha = need ? ex2(m_used - m_new) : 1.f;
 #pragma unroll
                     for (int ch = 0; ch < D / 32; ++ch) {
                         uint32_t o[32];
-                        tc::ld_32x32b_x32(tmem + lane_base + kColO + ch * 32, o);
+                        tc::ld_32x32b_x32(tmem + lane_base + col_o + ch * 32, o);
                         tc::wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tc::st_32x32b_x32(tmem + lane_base + kColO + ch * 32, o);
+                        tc::st_32x32b_x32(tmem + lane_base + col_o + ch * 32, o);
                     }
                     tc::wait_st();
                 }
@@ -388,28 +411,30 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                     l *= ex2(m_used - m_new);                     // ex2(-inf) = 0 on the first visible key
                     m_used = m_new;
                 }
-                const float mref = m_used == -INFINITY ? 0.f : m_used;
-                uint32_t pk[kBN / 2];
-                float lt = 0.f;
+                const float nref = m_used == -INFINITY ? 0.f : -m_used;
+                uint32_t pk[kHalfKeys / 2];
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < kBN / 2; ++i) {
-                    const float p0 = ex2(x[2 * i] - mref), p1 = ex2(x[2 * i + 1] - mref);
-                    lt += p0 + p1;
+                for (int i = 0; i < kHalfKeys / 2; ++i) {
+                    const float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), cs, nref));
+                    const float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), cs, nref));
+                    l4[i & 3] += p0 + p1;
                     pk[i] = pack_bf16x2(p0, p1);
                 }
-                l += lt;
-                // the single P buffer is free once O += P(j-1) V(j-1) is done
-                if (j >= 1 && !o_ready && !(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1)))
-                    break;
+                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                // P buffer j mod 2 was last read by O += P(j-2) V(j-2), which
+                // finished before S(j) (issued after it) was signalled
+                uint8_t *prow = pbuf + b * L::kPTile + r * 128;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int chunk = half * 4 + ch;
                     const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-                    *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = v4;
+                    *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) = v4;
                 }
                 fence_proxy_async();                             // generic writes -> tensor-core reads
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(p_full);
+                if (lane == 0) mbar_arrive(&p_full[b]);
                 first = false;
                 ++j;
                 if (mt.y & kMetaLast) break;
@@ -420,38 +445,63 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             if (has_tiles) {
                 if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
                 tc::fence_after_sync();
+                if (half == 1) {
+                    // publish this half's (m, l); the half-0 warp merges
+                    xml[r] = make_float2(m_used, l);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(xch);
+                    ++e;
+                    continue;
+                }
+                if (!(ok = wwait(xch, e & 1))) break;
+                ++e;
+            } else if (half == 1) {
+                continue;
+            }
+            // half-0 warps: merge the two halves and write
+            float s0 = 1.f, s1 = 0.f, M = m_used, Lt = l;
+            if (has_tiles) {
+                const float2 o1 = xml[r];
+                M = fmaxf(m_used, o1.x);
+                const float Mref = M == -INFINITY ? 0.f : M;
+                s0 = ex2(m_used - Mref);
+                s1 = ex2(o1.x - Mref);
+                Lt = l * s0 + o1.y * s1;
             }
             const bool whole = role == 0;
             const int slot = role == 1 ? 2 * c : 2 * c + 1;
             const int pr = qi * G + g;                            // row within the unit's G * Lq rows
             const long long tok = seg.s.q0 + qi;
             const int h = seg.hk * G + g;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
             if (has_tiles) {
 #pragma unroll
                 for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t o[32];
+                    uint32_t o0[32], o1[32];
                     __syncwarp();
-                    tc::ld_32x32b_x32(tmem + lane_base + kColO + ch * 32, o);   // warp-collective
+                    tc::ld_32x32b_x32(tmem + lane_base + kColO0 + ch * 32, o0);   // warp-collective
+                    tc::ld_32x32b_x32(tmem + lane_base + kColO1 + ch * 32, o1);
                     tc::wait_ld();
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o0[i]) * s0 + __uint_as_float(o1[i]) * s1;
                     if (!valid) {
                     } else if (whole) {
                         uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D + ch * 32);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
+                        for (int q4 = 0; q4 < 4; ++q4) {
                             uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-                            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-                            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-                            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-                            dst[v] = w;
+                            w.x = pack_bf16x2(v[8 * q4 + 0] * inv, v[8 * q4 + 1] * inv);
+                            w.y = pack_bf16x2(v[8 * q4 + 2] * inv, v[8 * q4 + 3] * inv);
+                            w.z = pack_bf16x2(v[8 * q4 + 4] * inv, v[8 * q4 + 5] * inv);
+                            w.w = pack_bf16x2(v[8 * q4 + 6] * inv, v[8 * q4 + 7] * inv);
+                            dst[q4] = w;
                         }
                     } else {
                         float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((long long)slot * kRows + pr) * D + ch * 32);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
                     }
                 }
                 tc::fence_before_sync();
@@ -460,16 +510,16 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             } else if (valid && whole) {
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D);
 #pragma unroll
-                for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                for (int q4 = 0; q4 < D / 8; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
             }
             if (valid) {
                 if (whole)
-                    p.lse[tok * p.Hq + h] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+                    p.lse[tok * p.Hq + h] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
                 else
-                    p.ml_part[(long long)slot * kRows + pr] = make_float2(m_used, l);
+                    p.ml_part[(long long)slot * kRows + pr] = make_float2(M, Lt);
             }
             // publish this warp's rows of the part (the combine waits for all
-            // kSoftWarps warps of each of the unit's n blocks)
+            // kEpiWarps writer warps of each of the unit's n blocks)
             if (!whole) {
                 __syncwarp();
                 if (lane == 0) red_add_release_gpu(p.done + (long long)seg.b * p.Hkv + seg.hk, 1u);
@@ -497,14 +547,19 @@ void *tc_kernel_ptr() {
 size_t tc_stage_bytes(int D) { return D == 64 ? TcLayout<64>::kStage : TcLayout<128>::kStage; }
 
 size_t tc_smem_bytes(int D, int stages) {
-    const size_t fixed = D == 64 ? 2 * TcLayout<64>::kQTile + TcLayout<64>::kPTile
-                                 : 2 * TcLayout<128>::kQTile + TcLayout<128>::kPTile;
-    // 1 KB alignment slack + ring + Q tiles + P tile + barriers + meta + scan + (first, T) + stop flag, tmem slot
-    return 1024 + tc_stage_bytes(D) * stages + fixed + (2 * stages + 14) * 8 + stages * 8 + (8 + 3) * 8 + 16;
+    const size_t fixed = D == 64 ? 2 * TcLayout<64>::kQTile + 2 * TcLayout<64>::kPTile
+                                 : 2 * TcLayout<128>::kQTile + 2 * TcLayout<128>::kPTile;
+    // 1 KB alignment slack + ring + Q tiles + P tiles + barriers + meta + half-1 (m, l) + scan +
+    // (first, T) + stop flag, tmem slot
+    const size_t need = 1024 + tc_stage_bytes(D) * stages + fixed + (2 * stages + 17) * 8 + stages * 8 +
+                        kRows * 8 + (kThreads / 32 + 3) * 8 + 16;
+    // at least half an SM's shared memory, so one block holds an SM and its
+    // tensor-memory allocation never waits for another block's
+    return need > kMinSmemBytes ? need : kMinSmemBytes;
 }
 
 int tc_rows() { return kRows; }
-int tc_parts_per_block() { return kSoftWarps; }
+int tc_parts_per_block() { return kEpiWarps; }
 
 cudaError_t tc_prepare(int D, int stages, int ctas) {
     void *fn = D == 64 ? tc_kernel_ptr<64>() : tc_kernel_ptr<128>();
