@@ -177,7 +177,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         ctas = std::min<long long>(ctas, std::max(1LL, max_tiles));
         ctas = std::min<long long>(ctas, 65535);
         d.ctas = (int)ctas;
-        auto smem_of = [&](int st) { return tcv ? tc_smem_bytes(D, st) : mma_smem_bytes(D, NT, st, d.ctas); };
+        auto smem_of = [&](int st) { return tcv ? tc_smem_need(D, st) : mma_smem_bytes(D, NT, st, d.ctas); };
         const size_t stage_bytes = tcv ? tc_stage_bytes(D) : mma_stage_bytes(D);
         int stages = o && o->stages ? o->stages : (int)((smem_block - smem_of(0)) / stage_bytes);
         stages = std::min(stages, 8);
@@ -185,7 +185,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         d.stages = stages;
         d.rows_per_block = tcv ? tc_rows() : 8 * NT;
         d.row_tiles = 1;
-        d.smem_bytes = (int)smem_of(stages);
+        d.smem_bytes = (int)(tcv ? tc_smem_bytes(D, stages) : smem_of(stages));
         merge_bytes = tcv ? 0 : (int)mma_merge_bytes(D, NT, d.ctas);
         d.nsplit = 0;
         d.chunk = 0;

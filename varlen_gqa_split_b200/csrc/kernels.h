@@ -31,7 +31,8 @@ cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUt
 // Persistent TMA-fed tcgen05 split kernel (accumulators in tensor memory),
 // up to tc_rows() query rows per KV head
 size_t tc_stage_bytes(int D);
-size_t tc_smem_bytes(int D, int stages);
+size_t tc_smem_need(int D, int stages);    // bytes the layout uses
+size_t tc_smem_bytes(int D, int stages);   // bytes requested at launch (>= half an SM)
 int tc_rows();
 int tc_parts_per_block();
 cudaError_t tc_prepare(int D, int stages, int ctas);

@@ -12,12 +12,12 @@
 //     O [128 rows x D]       += P [128 x 64 keys] . V        (P bf16 in shared memory, O in tensor memory)
 //
 // Warp roles (320 threads):
-//   warp 8, one lane -- producer: loads each unit's Q tile (one TMA box of G
+//   warp 9, one lane -- producer: loads each unit's Q tile (one TMA box of G
 //     heads x max_q tokens, right-aligned so it ends at the sequence's last
 //     query token; rows past the sequence's own tokens are never written)
 //     into one of two Q buffers, then streams the unit's K and V tiles into a
 //     ring of shared-memory stages exactly like the warp-MMA kernel;
-//   warp 9, one lane -- MMA issuer: S(j) = Q K_j^T into one of two S buffers,
+//   warp 8, one lane -- MMA issuer: S(j) = Q K_j^T into one of two S buffers,
 //     then O += P(j-1) V_{j-1}, so the softmax of tile j overlaps the second
 //     product of tile j-1 (a unit's last tile is not held back: its second
 //     product follows at once); completion is tracked with tcgen05.commit on
@@ -31,8 +31,8 @@
 //     the epilogue merges the two halves like two split-KV partials.  The
 //     scores are masked (keys before the tile's own start when the tile was
 //     right-aligned, and keys past Lk - Lq + qi under the tail-aligned causal
-//     mask), and P is written as bf16 into one of two P buffers in the
-//     128-byte swizzled operand layout.
+//     mask), and P is written as bf16 pairs into one of two P buffers in
+//     tensor memory, from where the second product reads its A operand.
 //
 // The running max is rescaled lazily: O_h in tensor memory is multiplied by
 // 2^(m_old - m_new) only when a row's max grows by more than 2^8 (rare after
@@ -59,15 +59,16 @@ using namespace sched;
 constexpr int kRows = 128;                // MMA M: query rows of a unit
 constexpr int kSoftWarps = 8;             // two per tensor-memory lane quarter (column halves)
 constexpr int kEpiWarps = 4;              // the half-0 warps write the outputs
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 8;              // sub-partition 0: its rows are the last to hold query rows
+constexpr int kProducerWarp = 9;
 constexpr int kThreads = 320;
 constexpr int kHalfKeys = kBN / 2;
 constexpr int kMetaLast = 1;              // stage flag: the block's last tile of the unit
 constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends here
 constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold (base-2 units)
-constexpr uint32_t kTmemCols = 512;       // S buffers [0, 128), O_0 [128, 128 + D), O_1 [256, 256 + D)
-constexpr uint32_t kColS = 0, kColO0 = 128, kColO1 = 256;
+constexpr uint32_t kTmemCols = 512;       // S [0, 128), O_0 [128, 128 + D), O_1 [256, 256 + D), P [384, 448)
+constexpr uint32_t kColS = 0, kColO0 = 128, kColO1 = 256, kColP = 384;
+constexpr uint32_t kPCols = kBN / 2;      // bf16 pairs of one P buffer
 constexpr size_t kMinSmemBytes = 120 * 1024;
 
 template <int D>
@@ -78,7 +79,6 @@ struct TcLayout {
     static constexpr int kStage = 2 * kKvTile;              // K + V
     static constexpr int kQRegion = kRows * 128;            // 128 rows x 128 B
     static constexpr int kQTile = kHalves * kQRegion;
-    static constexpr int kPTile = kRows * 128;              // 128 rows x 64 keys bf16
 };
 
 // bounded mbarrier wait that also gives up when another role raised the stop flag
@@ -106,8 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;                                    // [stages][K tile | V tile]
     uint8_t *qbuf = ring + stages * L::kStage;               // [2][Q tile]
-    uint8_t *pbuf = qbuf + 2 * L::kQTile;                    // [2][P tile]
-    uint64_t *full = reinterpret_cast<uint64_t *>(pbuf + 2 * L::kPTile);
+    uint64_t *full = reinterpret_cast<uint64_t *>(qbuf + 2 * L::kQTile);
     uint64_t *empty = full + stages;
     uint64_t *q_full = empty + stages;       // [2] Q tile landed
     uint64_t *q_free = q_full + 2;           // [2] last product reading the Q tile done
@@ -238,8 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         if (lane == 0) {
             constexpr uint32_t kIdS = tc::idesc_bf16_f32(kRows, kBN, false);
             constexpr uint32_t kIdO = tc::idesc_bf16_f32(kRows, D, true);
-            const uint32_t ring0 = smem_u32(ring), q0 = smem_u32(qbuf), p0 = smem_u32(pbuf);
-            int j = 0, st = 0, k = 0, e = 0;
+            const uint32_t ring0 = smem_u32(ring), q0 = smem_u32(qbuf);
+            int j = 0, k = 0, e = 0, s = 0;
+            uint32_t sph = 0;                       // ring position and phase
             bool have_prev = false, ok = true;
             int pj = 0, ps = 0, pe = 0;
             bool pfirst = false;
@@ -250,16 +250,15 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 if (!wait_bar(&p_full[pj & 1], (pj >> 1) & 1, stop, p)) return false;
                 if (pfirst && pe >= 1 && !wait_bar(o_free, (pe - 1) & 1, stop, p)) return false;
                 tc::fence_after_sync();
-                const uint32_t v0 = ring0 + ps * L::kStage + L::kKvTile;
-                const uint32_t pa = p0 + (pj & 1) * L::kPTile;
+                const uint64_t v0 = tc::smem_desc_sw128(ring0 + ps * L::kStage + L::kKvTile, L::kKvRegion, 1024);
+                const uint32_t pa = tmem + kColP + (pj & 1) * kPCols;
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int kk = 0; kk < kHalfKeys / 16; ++kk) {
                         const int key = h * kHalfKeys + kk * 16;
-                        const uint64_t a = tc::smem_desc_sw128(pa + key * 2, 16, 1024);
-                        const uint64_t b = tc::smem_desc_sw128(v0 + key * 128, L::kKvRegion, 1024);
-                        tc::mma_bf16_ss(tmem + (h ? kColO1 : kColO0), a, b, kIdO, !pfirst || kk > 0);
+                        tc::mma_bf16_ts(tmem + (h ? kColO1 : kColO0), pa + key / 2, v0 + ((key * 128) >> 4), kIdO,
+                                        !pfirst || kk > 0);
                     }
                 tc::commit(smem_u32(&empty[ps]));
                 tc::commit(smem_u32(&o_done[pj & 1]));
@@ -275,32 +274,37 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 const uint32_t qa = q0 + qb * L::kQTile;
                 bool first = true;
                 while (true) {
-                    const int s = st % stages;
-                    if (!(ok = wait_bar(&full[s], (st / stages) & 1, stop, p))) break;
+                    if (!(ok = wait_bar(&full[s], sph, stop, p))) break;
                     const int2 mt = meta[s];
-                    ++st;
+                    const int cs_ = s;
+                    if (++s == stages) {
+                        s = 0;
+                        sph ^= 1;
+                    }
                     if (mt.y & kMetaEmpty) {            // the unit ends without a tile here
-                        mbar_arrive(&empty[s]);
+                        mbar_arrive(&empty[cs_]);
                         mbar_arrive(&q_free[qb]);
                         break;
                     }
                     const int b = j & 1;
                     if (j >= 2 && !(ok = wait_bar(&s_free[b], ((j - 2) >> 1) & 1, stop, p))) break;
                     tc::fence_after_sync();
-                    const uint32_t k0 = ring0 + s * L::kStage;
+                    // descriptors advance by adding (byte offset >> 4) to the
+                    // start-address field (shared addresses stay below 2^18)
+                    const uint64_t a0 = tc::smem_desc_sw128(qa, 16, 1024);
+                    const uint64_t b0 = tc::smem_desc_sw128(ring0 + cs_ * L::kStage, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const int hf = kk >> 2, cc = (kk & 3) * 32;
-                        const uint64_t a = tc::smem_desc_sw128(qa + hf * L::kQRegion + cc, 16, 1024);
-                        const uint64_t bd = tc::smem_desc_sw128(k0 + hf * L::kKvRegion + cc, 16, 1024);
-                        tc::mma_bf16_ss(tmem + kColS + b * kBN, a, bd, kIdS, kk > 0);
+                        tc::mma_bf16_ss(tmem + kColS + b * kBN, a0 + ((hf * L::kQRegion + cc) >> 4),
+                                        b0 + ((hf * L::kKvRegion + cc) >> 4), kIdS, kk > 0);
                     }
                     tc::commit(smem_u32(&s_full[b]));
                     if (mt.y & kMetaLast) tc::commit(smem_u32(&q_free[qb]));
                     if (have_prev && !(ok = issue_pv())) break;
                     have_prev = true;
                     pj = j;
-                    ps = s;
+                    ps = cs_;
                     pfirst = first;
                     pe = e;
                     first = false;
@@ -337,7 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const bool w = wait_bar(bar, parity, stop, p);
             return __all_sync(0xffffffffu, w);
         };
-        int j = 0, st = 0, e = 0;
+        int j = 0, e = 0, s = 0;
+        uint32_t sph = 0;                           // ring position and phase
         bool ok = true;
         OrderedWalker wk;
         wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
@@ -349,19 +354,35 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const int qi = tq - (QT - Lq);                       // this row's query token in the sequence
             const bool valid = tq < QT && qi >= 0;
             const int vis = valid ? Lk - Lq + qi + 1 : 0;        // keys [0, vis) visible (tail-aligned causal)
+            // a warp none of whose 32 rows is a query row of this unit only
+            // keeps the barrier protocol (its P rows feed O rows nobody reads)
+            const bool act = __any_sync(0xffffffffu, valid);
             float m_used = -INFINITY, l = 0.f;
             bool first = true, has_tiles = false;
             while (true) {
-                const int s = st % stages;
-                if (!(ok = wwait(&full[s], (st / stages) & 1))) break;
+                if (!(ok = wwait(&full[s], sph))) break;
                 const int2 mt = meta[s];
-                ++st;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
+                if (++s == stages) {
+                    s = 0;
+                    sph ^= 1;
+                }
                 if (mt.y & kMetaEmpty) break;
                 has_tiles = true;
                 const int b = j & 1;
                 if (!(ok = wwait(&s_full[b], (j >> 1) & 1))) break;
+                if (!act) {
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&s_free[b]);
+                        mbar_arrive(&p_full[b]);
+                    }
+                    first = false;
+                    ++j;
+                    if (mt.y & kMetaLast) break;
+                    continue;
+                }
                 tc::fence_after_sync();
                 uint32_t sv[kHalfKeys];
                 tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kBN + half * kHalfKeys, sv);
@@ -424,14 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
                 // P buffer j mod 2 was last read by O += P(j-2) V(j-2), which
                 // finished before S(j) (issued after it) was signalled
-                uint8_t *prow = pbuf + b * L::kPTile + r * 128;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int chunk = half * 4 + ch;
-                    const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-                    *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) = v4;
-                }
-                fence_proxy_async();                             // generic writes -> tensor-core reads
+                tc::st_32x32b_x16(tmem + lane_base + kColP + b * kPCols + half * (kHalfKeys / 2), pk);
+                tc::wait_st();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[b]);
@@ -477,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             if (has_tiles) {
 #pragma unroll
                 for (int ch = 0; ch < D / 32; ++ch) {
+                    if (!act) break;
                     uint32_t o0[32], o1[32];
                     __syncwarp();
                     tc::ld_32x32b_x32(tmem + lane_base + kColO0 + ch * 32, o0);   // warp-collective
@@ -546,15 +562,18 @@ void *tc_kernel_ptr() {
 
 size_t tc_stage_bytes(int D) { return D == 64 ? TcLayout<64>::kStage : TcLayout<128>::kStage; }
 
-size_t tc_smem_bytes(int D, int stages) {
-    const size_t fixed = D == 64 ? 2 * TcLayout<64>::kQTile + 2 * TcLayout<64>::kPTile
-                                 : 2 * TcLayout<128>::kQTile + 2 * TcLayout<128>::kPTile;
-    // 1 KB alignment slack + ring + Q tiles + P tiles + barriers + meta + half-1 (m, l) + scan +
+size_t tc_smem_need(int D, int stages) {
+    const size_t fixed = D == 64 ? 2 * TcLayout<64>::kQTile : 2 * TcLayout<128>::kQTile;
+    // 1 KB alignment slack + ring + Q tiles + barriers + meta + half-1 (m, l) + scan +
     // (first, T) + stop flag, tmem slot
-    const size_t need = 1024 + tc_stage_bytes(D) * stages + fixed + (2 * stages + 17) * 8 + stages * 8 +
-                        kRows * 8 + (kThreads / 32 + 3) * 8 + 16;
+    return 1024 + tc_stage_bytes(D) * stages + fixed + (2 * stages + 17) * 8 + stages * 8 + kRows * 8 +
+           (kThreads / 32 + 3) * 8 + 16;
+}
+
+size_t tc_smem_bytes(int D, int stages) {
     // at least half an SM's shared memory, so one block holds an SM and its
     // tensor-memory allocation never waits for another block's
+    const size_t need = tc_smem_need(D, stages);
     return need > kMinSmemBytes ? need : kMinSmemBytes;
 }
 
