@@ -179,7 +179,11 @@ def recorded_traffic(workload: str, kernel: str):
 
 # ------------------------------------------------------------------ distributed
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun env).  The ranks run independent
+    replicas of the workload; the only collectives are the barrier around the
+    timed region and the max of the ranks' times.  backend="gloo" runs the
+    same logic on CPU (tests)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -189,9 +193,12 @@ def dist_setup(n_gpus: int):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
         pg = dist
     return rank, world, local, pg
 
@@ -199,7 +206,8 @@ def dist_setup(n_gpus: int):
 def max_over_ranks(x: float, pg) -> float:
     if pg is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 
