@@ -93,6 +93,17 @@ int encode_q_map(CUtensorMap *map, const void *base, int Hq, int D, int G, int m
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+int gcd(int a, int b) { return b ? gcd(b, a % b) : a; }
+
+// A stride near n / golden ratio that is coprime with n: b -> (b * stride)
+// mod n is then a permutation of the blocks that scatters neighbours.
+int share_stride(int n) {
+    if (n <= 2) return 1;
+    for (int s = (int)(n * 0.6180339887) | 1; s > 1; --s)
+        if (gcd(s, n) == 1) return s;
+    return 1;
+}
+
 bool aligned(const void *ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
 }  // namespace
@@ -355,6 +366,7 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
     p.fused = d.combine == ATTN_COMBINE_FUSED;
     p.merge_bytes = plan->merge_bytes;
     p.ctas_max = d.ctas;
+    p.share_stride = share_stride(d.ctas);
     const bool persistent = d.variant == ATTN_VARIANT_MMA || d.variant == ATTN_VARIANT_TC;
     p.dynamic = persistent && !d.deterministic;
     p.done_per_part = d.variant == ATTN_VARIANT_TC ? tc_parts_per_block() : 1;

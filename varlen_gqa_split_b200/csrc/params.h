@@ -33,6 +33,7 @@ struct Params {
     int ctas_max;              // tensor-core path: blocks of the launch (merge table size)
     int dynamic;               // tensor-core path: blocks sharing a cut unit claim its tiles
     int done_per_part;         // tensor-core path: releases on `done` per written part
+    int share_stride;          // tensor-core path: block b takes share (b * share_stride) mod blocks
 };
 
 }  // namespace vgqa

@@ -126,7 +126,10 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x;
+    // the block's share: consecutive blocks (which the hardware tends to
+    // place on neighbouring SMs) take shares far apart, so every unit shared
+    // by several blocks gets a mix of SMs rather than one neighbourhood
+    const int c = (int)(((long long)blockIdx.x * p.share_stride) % gridDim.x);
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
