@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
     constexpr int kCols = D / 4;
     constexpr int kT = 128;
     constexpr int kBatch = 12;             // loads in flight per thread (register budget)
+    constexpr int kFewParts = 4;           // up to this many parts: item-batched merge
+    constexpr int kItems = 3;              // items per thread per pass in the item-batched merge
     extern __shared__ __align__(16) uint8_t csm[];
     __shared__ long long scan[kT / 32];
     __shared__ long long first[3];
@@ -102,8 +104,71 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
     __syncthreads();
     if (!ok_flag) return;
 
-    // two threads per item (row, 4 columns), each merging every other part
-    // with a running max, kBatch loads in flight; the pair then combines
+    auto write_row = [&](int r, int d4, float Mt, float Lt, float4 acc) {
+        const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+        const int qi = r / G, h = seg.hk * G + r % G;
+        const long long tok = seg.s.q0 + qi;
+        uint2 pk;
+        pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2 *>(p.out + (tok * p.Hq + h) * D + d4) = pk;
+        if (d4 == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
+    };
+    if (n <= kFewParts) {
+        // few parts: one thread per item, kItems items per pass with all
+        // their loads in flight (the merge is latency-bound)
+        const int n_items = it_hi - it_lo;
+        for (int base = 0; base < n_items; base += kT * kItems) {
+            float2 ml[kItems][kFewParts];
+            float4 o[kItems][kFewParts];
+#pragma unroll
+            for (int i = 0; i < kItems; ++i) {
+                const int w = base + i * kT + tid;
+                const int it = it_lo + (w < n_items ? w : 0);
+                const int r = it / kCols, d4 = (it % kCols) * 4;
+#pragma unroll
+                for (int j = 0; j < kFewParts; ++j) {
+                    if (j < n && w < n_items) {
+                        const long long sl = slots[j];
+                        ml[i][j] = __ldcg(p.ml_part + sl * ROWS + r);
+                        o[i][j] = __ldcg(reinterpret_cast<const float4 *>(p.o_part + (sl * ROWS + r) * D + d4));
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kItems; ++i) {
+                const int w = base + i * kT + tid;
+                if (w >= n_items) continue;
+                const int it = it_lo + w;
+                float M = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < kFewParts; ++j)
+                    if (j < n && ml[i][j].y > 0.f) M = fmaxf(M, ml[i][j].x);
+                const float Mref = M == -INFINITY ? 0.f : M;
+                float L = 0.f;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < kFewParts; ++j) {
+                    if (j < n && ml[i][j].y > 0.f) {
+                        const float wq = ex2(ml[i][j].x - Mref);
+                        acc.x = fmaf(wq, o[i][j].x, acc.x);
+                        acc.y = fmaf(wq, o[i][j].y, acc.y);
+                        acc.z = fmaf(wq, o[i][j].z, acc.z);
+                        acc.w = fmaf(wq, o[i][j].w, acc.w);
+                        L = fmaf(wq, ml[i][j].y, L);
+                    }
+                }
+                write_row(it / kCols, (it % kCols) * 4, M, L, acc);
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && atomicAdd(p.done + u, 1u) == parts_done + (uint32_t)(nb - 1)) p.done[u] = 0u;
+        return;
+    }
+
+    // many parts: two threads per item (row, 4 columns), each merging every
+    // other part with a running max, kBatch loads in flight; the pair then
+    // combines
     const int n_work = 2 * (it_hi - it_lo);
     for (int base = 0; base < n_work; base += kT) {
         const int w = base + tid;
@@ -152,15 +217,9 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
             const float Mt = fmaxf(M, M2);
             const float Mref = Mt == -INFINITY ? 0.f : Mt;
             const float s1 = ex2(M - Mref), s2 = ex2(M2 - Mref);
-            const float Lt = L * s1 + L2 * s2;
-            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
-            const int qi = r / G, h = seg.hk * G + r % G;
-            const long long tok = seg.s.q0 + qi;
-            uint2 pk;
-            pk.x = pack_bf16x2((acc.x * s1 + a2.x * s2) * inv, (acc.y * s1 + a2.y * s2) * inv);
-            pk.y = pack_bf16x2((acc.z * s1 + a2.z * s2) * inv, (acc.w * s1 + a2.w * s2) * inv);
-            *reinterpret_cast<uint2 *>(p.out + (tok * p.Hq + h) * D + d4) = pk;
-            if (d4 == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
+            write_row(r, d4, Mt, L * s1 + L2 * s2,
+                      make_float4(acc.x * s1 + a2.x * s2, acc.y * s1 + a2.y * s2, acc.z * s1 + a2.z * s2,
+                                  acc.w * s1 + a2.w * s2));
         }
     }
     __syncthreads();
@@ -182,9 +241,9 @@ cudaError_t combine_slots_prepare(int D, int ctas) {
 }
 
 int combine_slots_split(int rows, int D) {
-    // about 512 (row, 4-column) items per block at most, up to 8 blocks per slot
+    // about 1024 (row, 4-column) items per block at most, up to 8 blocks per slot
     const int items = rows * (D / 4);
-    const int S = (items + 511) / 512;
+    const int S = (items + 1023) / 1024;
     return S < 1 ? 1 : (S > 8 ? 8 : S);
 }
 
