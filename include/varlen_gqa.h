@@ -187,6 +187,29 @@ int attn_run(attn_plan_t plan, const void *q, const void *k, const void *v,
              void *stream);
 
 /*
+ * attn_run_strided -- attn_run with K and V as views into larger buffers.
+ *
+ *   k_token_stride, v_token_stride  elements between consecutive tokens of
+ *          k and v; within a token the Hkv heads of D elements stay
+ *          contiguous.  Each stride is >= Hkv * D, a multiple of 8 (16-byte
+ *          rows) and at most 2^38; otherwise ATTN_E_INVALID_ARG and nothing is
+ *          launched.  A fused cache laid out [T, 2, Hkv, D] passes k = base,
+ *          v = base + Hkv * D and both strides 2 * Hkv * D.  All other
+ *          arguments, the outputs and the error behaviour are those of
+ *          attn_run (which is this call with both strides Hkv * D).
+ *
+ * Source: the declared-stride contract of THD inputs instead of a packed-
+ * stride assumption, cudnn-frontend issue #552 "frost(sdpa): THD execute host
+ * round-trip", section Related (#538, #539); stride parameters in the split
+ * kernel's interface, magik.net "Wiring Split-K Dispatch into a Custom CUDA
+ * Attention Kernel", section "The Message".  Not planned separately: one plan
+ * serves packed and strided calls.
+ */
+int attn_run_strided(attn_plan_t plan, const void *q, const void *k, const void *v,
+                     const int32_t *cu_q, const int32_t *cu_k, void *out, float *lse,
+                     int64_t k_token_stride, int64_t v_token_stride, void *stream);
+
+/*
  * attn_check_error -- synchronise `stream`, then read and clear the plan's
  * sticky device error bits (ATTN_DEV_ERR_*) into *flags.  When a bit was set
  * it also resets the plan's merge tickets, so the plan stays usable after a

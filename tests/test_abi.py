@@ -32,8 +32,8 @@ def libvgqa():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_check_error",
-              "attn_destroy", "attn_strerror"):
+    for n in ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_run_strided", "attn_check_error",
+              "attn_destroy", "attn_strerror", "attn_run_noalloc"):
         assert n in names
 
 
@@ -72,6 +72,8 @@ def test_strerror_and_host_errors_without_gpu(libvgqa):
     assert lib.attn_plan(ctypes.byref(h), 2, 128, 4, 1, 96, 1) == -2       # head dim
     lib.attn_run.argtypes = [ctypes.c_void_p] * 9
     assert lib.attn_run(None, None, None, None, None, None, None, None, None) == -5
+    lib.attn_run_strided.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
+    assert lib.attn_run_strided(None, None, None, None, None, None, None, None, 1024, 1024, None) == -5
     lib.attn_plan_info.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     buf = ctypes.create_string_buffer(256)
     assert lib.attn_plan_info(ctypes.c_void_p(0x1234), buf) == -5          # unknown handle

@@ -223,6 +223,64 @@ def test_dynamic_balance_repeats_within_rounding():
         assert (o.float() - runs[0][0].float()).abs().max().item() <= 2 * ATOL_OUT
 
 
+# ------------------------------------------------------------ strided K/V (views into larger buffers)
+
+@pytest.mark.parametrize("variant,Hq,max_q", [(MMA, 16, 1), (TC, 32, 8), (SIMT, 16, 2)])
+@pytest.mark.parametrize("layout", ["fused_kv", "wide_heads"])
+def test_strided_kv_views(variant, Hq, max_q, layout):
+    """K and V as views with a token stride: the halves of a fused [T, 2, Hkv, D]
+    cache, or Hkv heads out of a buffer with more heads per token.  The
+    oracle gets packed copies of the same bytes."""
+    Hkv, D = 4, 128
+    rng = np.random.default_rng(17)
+    B = 7
+    lq = rng.integers(1, max_q, B, endpoint=True)
+    lk = rng.integers(0, 600, B)
+    lk[0] = 0
+    sh = W.Shape("strided", B=B + 1, Hq=Hq, Hkv=Hkv, D=D, max_q=max_q, s_max=600)
+    batch = W.make_batch(sh, lq, lk, seed=23, gen_device="cuda")
+    T = batch.k.shape[0]
+    if layout == "fused_kv":
+        buf = torch.empty(T, 2, Hkv, D, dtype=torch.bfloat16, device="cuda")
+        buf[:, 0] = batch.k
+        buf[:, 1] = batch.v
+        kv, vv = buf[:, 0], buf[:, 1]
+    else:
+        buf_k = torch.zeros(T, Hkv + 3, D, dtype=torch.bfloat16, device="cuda")
+        buf_v = torch.zeros(T, Hkv + 5, D, dtype=torch.bfloat16, device="cuda")
+        buf_k[:, 2:2 + Hkv] = batch.k
+        buf_v[:, 1:1 + Hkv] = batch.v
+        kv, vv = buf_k[:, 2:2 + Hkv], buf_v[:, 1:1 + Hkv]
+    assert not kv.is_contiguous()
+    plan = plan_for(sh, variant=variant)
+    q = batch.q.cuda()
+    cu_q = torch.from_numpy(batch.cu_q).cuda()
+    cu_k = torch.from_numpy(batch.cu_k).cuda()
+    out = sentinel_out(q.shape[0], Hq, D)
+    lse = sentinel_lse(q.shape[0], Hq)
+    plan.run(q, kv, vv, cu_q, cu_k, out, lse)
+    torch.cuda.synchronize()
+    assert plan.check_error() == 0
+    ref_o, ref_l = oracle_full(batch)
+    compare_full(out.cpu(), lse.cpu(), ref_o, ref_l, covered_rows(batch))
+
+
+def test_strided_kv_rejects_bad_strides():
+    import ctypes
+    sh = W.Shape("strided_bad", B=2, Hq=8, Hkv=2, D=64, max_q=1, s_max=64)
+    plan = plan_for(sh)
+    lib = vg.lib()
+    t = torch.zeros(256, dtype=torch.bfloat16, device="cuda")
+    cu = torch.zeros(3, dtype=torch.int32, device="cuda")
+    lse = torch.zeros(16, dtype=torch.float32, device="cuda")
+    args = [plan._h, t.data_ptr(), t.data_ptr(), t.data_ptr(), cu.data_ptr(), cu.data_ptr(), t.data_ptr(),
+            lse.data_ptr()]
+    for ks, vs in ((64, 128), (128, 132), (128, 1 << 40)):       # below Hkv*D, not a multiple of 8, too large
+        assert lib.attn_run_strided(*args, ks, vs, None) == -1     # ATTN_E_INVALID_ARG
+    assert lib.attn_run_strided(*args, 136, 128, None) == 0        # wider, aligned: accepted
+    torch.cuda.synchronize()
+
+
 # ------------------------------------------------------------ placement and edge cases
 
 def _packed_cases(B, values):

@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.attn_plan_info.restype = i
         L.attn_run.argtypes = [vp, vp, vp, vp, i32p, i32p, vp, vp, vp]
         L.attn_run.restype = i
+        L.attn_run_strided.argtypes = [vp, vp, vp, vp, i32p, i32p, vp, vp, ctypes.c_int64, ctypes.c_int64, vp]
+        L.attn_run_strided.restype = i
         L.attn_check_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.attn_check_error.restype = i
         L.attn_destroy.argtypes = [vp]
@@ -133,20 +135,26 @@ class Plan:
     def run(self, q, k, v, cu_q, cu_k, out=None, lse=None, stream=None):
         """out, lse = plan.run(q, k, v, cu_q, cu_k[, out, lse, stream]).
 
-        q [T_q, Hq, D], k / v [T_kv, Hkv, D] bf16 contiguous CUDA tensors;
+        q [T_q, Hq, D] bf16 contiguous CUDA tensor; k / v [T_kv, Hkv, D] bf16
+        CUDA tensors whose heads are contiguous within a token -- packed, or
+        views into a larger buffer with a token stride (e.g. the halves of a
+        fused [T, 2, Hkv, D] cache), which go through attn_run_strided;
         cu_q / cu_k int32 CUDA tensors with B_max + 1 entries; out / lse are
         allocated when not given (pass them for graph capture)."""
         if self._h is None:
             raise AttnError(-5, "attn_run")
         i = self.info
-        for name, t in (("q", q), ("k", k), ("v", v)):
-            if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-                raise TypeError(f"{name} must be a contiguous bf16 CUDA tensor")
+        if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
+            raise TypeError("q must be a contiguous bf16 CUDA tensor")
         if q.dim() != 3 or q.shape[1:] != (i["Hq"], i["D"]):
             raise ValueError(f"q must be [T_q, {i['Hq']}, {i['D']}]")
         for name, t in (("k", k), ("v", v)):
+            if t.dtype != torch.bfloat16 or not t.is_cuda:
+                raise TypeError(f"{name} must be a bf16 CUDA tensor")
             if t.dim() != 3 or t.shape[1:] != (i["Hkv"], i["D"]):
                 raise ValueError(f"{name} must be [T_kv, {i['Hkv']}, {i['D']}]")
+            if t.stride(2) != 1 or t.stride(1) != i["D"] or (t.shape[0] > 1 and t.stride(0) < i["Hkv"] * i["D"]):
+                raise ValueError(f"{name} must keep each token's heads contiguous (strides (s, D, 1), s >= Hkv*D)")
         for name, t in (("cu_q", cu_q), ("cu_k", cu_k)):
             if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.numel() != i["B_max"] + 1:
                 raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of B_max+1 entries")
@@ -158,9 +166,18 @@ class Plan:
             raise ValueError("out must be a contiguous bf16 tensor shaped like q")
         if lse.dtype != torch.float32 or lse.shape != (q.shape[0], i["Hq"]) or not lse.is_contiguous():
             raise ValueError("lse must be a contiguous fp32 tensor [T_q, Hq]")
-        rc = lib().attn_run(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_q.data_ptr(),
-                            cu_k.data_ptr(), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
-        _check(rc, "attn_run")
+        packed = i["Hkv"] * i["D"]
+        ks = k.stride(0) if k.shape[0] > 1 else packed
+        vs = v.stride(0) if v.shape[0] > 1 else packed
+        if ks == packed and vs == packed:
+            rc = lib().attn_run(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_q.data_ptr(),
+                                cu_k.data_ptr(), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
+            _check(rc, "attn_run")
+        else:
+            rc = lib().attn_run_strided(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_q.data_ptr(),
+                                        cu_k.data_ptr(), out.data_ptr(), lse.data_ptr(), ks, vs,
+                                        _stream_ptr(stream))
+            _check(rc, "attn_run_strided")
         return out, lse
 
     def check_error(self, stream=None) -> int:

@@ -65,9 +65,9 @@ int get_encoder() {
 // swizzle.  The token extent is left open (2^31 - 1): every load the kernel
 // issues ends at or before its sequence's last key (cu_k[b+1] - 1), so the
 // real buffer length never enters.
-int encode_kv_map(CUtensorMap *map, const void *base, int Hkv, int D, int block_n) {
+int encode_kv_map(CUtensorMap *map, const void *base, int Hkv, int D, int block_n, long long token_stride) {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)0x7fffffff};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)token_stride * 2};
     cuuint32_t box[3] = {64, 1, (cuuint32_t)block_n};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
@@ -325,8 +325,10 @@ ATTN_EXPORT int attn_plan_info(attn_plan_t plan, attn_plan_desc *desc) {
     return ATTN_OK;
 }
 
-ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const void *v, const int32_t *cu_q,
-                         const int32_t *cu_k, void *out, float *lse, void *stream) {
+namespace {
+
+int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, const int32_t *cu_q,
+             const int32_t *cu_k, void *out, float *lse, long long k_stride, long long v_stride, void *stream) {
     if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
     if (!q || !k || !v || !cu_q || !cu_k || !out || !lse) return ATTN_E_NULL;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
@@ -360,6 +362,8 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
     p.rows_per_block = d.rows_per_block;
     p.row_tiles = d.row_tiles;
     p.scale_log2 = plan->scale_log2;
+    p.k_stride = k_stride;
+    p.v_stride = v_stride;
     p.ticket = plan->ticket;
     p.claim = reinterpret_cast<unsigned long long *>(plan->ticket);
     p.done = plan->ticket + 2 * (size_t)d.B_max * d.Hkv;
@@ -376,15 +380,15 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
     cudaError_t e;
     if (d.variant == ATTN_VARIANT_MMA) {
         CUtensorMap tm_k, tm_v;
-        if (encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n) != ATTN_OK ||
-            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n) != ATTN_OK)
+        if (encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n, k_stride) != ATTN_OK ||
+            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n, v_stride) != ATTN_OK)
             return ATTN_E_CUDA;
         e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, d.ctas, s);
     } else if (d.variant == ATTN_VARIANT_TC) {
         CUtensorMap tm_q, tm_k, tm_v;
         if (encode_q_map(&tm_q, q, d.Hq, d.D, d.G, d.max_q) != ATTN_OK ||
-            encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n) != ATTN_OK ||
-            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n) != ATTN_OK)
+            encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n, k_stride) != ATTN_OK ||
+            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n, v_stride) != ATTN_OK)
             return ATTN_E_CUDA;
         e = launch_split_tc(p, tm_q, tm_k, tm_v, d.stages, d.ctas, s);
     } else {
@@ -396,6 +400,27 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
         if (e != cudaSuccess) return ATTN_E_CUDA;
     }
     return ATTN_OK;
+}
+
+}  // namespace
+
+ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const void *v, const int32_t *cu_q,
+                         const int32_t *cu_k, void *out, float *lse, void *stream) {
+    if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
+    const long long packed = (long long)plan->d.Hkv * plan->d.D;
+    return run_impl(plan, q, k, v, cu_q, cu_k, out, lse, packed, packed, stream);
+}
+
+ATTN_EXPORT int attn_run_strided(attn_plan_t plan, const void *q, const void *k, const void *v,
+                                 const int32_t *cu_q, const int32_t *cu_k, void *out, float *lse,
+                                 int64_t k_token_stride, int64_t v_token_stride, void *stream) {
+    if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
+    const long long packed = (long long)plan->d.Hkv * plan->d.D;
+    // a token's heads stay contiguous; the token stride keeps 16-byte
+    // alignment (the tensor-map rule) and fits the tensor map's range
+    for (long long st : {(long long)k_token_stride, (long long)v_token_stride})
+        if (st < packed || st % 8 != 0 || st > (1ll << 38)) return ATTN_E_INVALID_ARG;
+    return run_impl(plan, q, k, v, cu_q, cu_k, out, lse, k_token_stride, v_token_stride, stream);
 }
 
 ATTN_EXPORT int attn_check_error(attn_plan_t plan, void *stream, uint32_t *flags) {

@@ -169,6 +169,7 @@ ATTN_EXPORT int attn_run_noalloc(int B_max, int s_max, int Hq, int Hkv, int D, i
     p.rows_per_block = kSimtRowsPerBlock;
     p.row_tiles = row_tiles;
     p.scale_log2 = (float)((1.0 / std::sqrt((double)D)) * 1.4426950408889634);
+    p.k_stride = p.v_stride = (long long)Hkv * D;
     p.fused = nsplit > 1;
     const dim3 grid(nsplit, Hkv * row_tiles, B_max);
     if (launch_split_simt(p, grid, st) != cudaSuccess) return ATTN_E_CUDA;

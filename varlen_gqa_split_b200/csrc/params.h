@@ -10,8 +10,8 @@ namespace vgqa {
 // Everything a split / combine launch needs.  Passed by value.
 struct Params {
     const __nv_bfloat16 *q;    // [T_q, Hq, D]
-    const __nv_bfloat16 *k;    // [T_kv, Hkv, D]
-    const __nv_bfloat16 *v;    // [T_kv, Hkv, D]
+    const __nv_bfloat16 *k;    // [T_kv, Hkv, D], token stride k_stride elements
+    const __nv_bfloat16 *v;    // [T_kv, Hkv, D], token stride v_stride elements
     const int32_t *cu_q;       // [B_max + 1]
     const int32_t *cu_k;       // [B_max + 1]
     __nv_bfloat16 *out;        // [T_q, Hq, D]
@@ -34,6 +34,8 @@ struct Params {
     int dynamic;               // tensor-core path: blocks sharing a cut unit claim its tiles
     int done_per_part;         // tensor-core path: releases on `done` per written part
     int share_stride;          // tensor-core path: block b takes share (b * share_stride) mod blocks
+    long long k_stride;        // elements between consecutive tokens of k (Hkv * D when packed)
+    long long v_stride;        // elements between consecutive tokens of v
 };
 
 }  // namespace vgqa

@@ -89,9 +89,10 @@ __global__ void __launch_bounds__(kThreads) split_simt_kernel(const Params p) {
             const int rr = c / kChunks, ch = c % kChunks;
             const int j = t0 + rr;
             const bool ok = j < kv_lim;
-            const long long off = ok ? ((long long)(k0 + j) * p.Hkv + hk) * D + ch * 8 : 0;
-            cp_async_16(smem_u32(&sm.k[buf][rr][ch * 8]), p.k + off, ok);
-            cp_async_16(smem_u32(&sm.v[buf][rr][ch * 8]), p.v + off, ok);
+            const long long tok = ok ? (long long)(k0 + j) : 0;
+            const long long hd = (long long)hk * D + ch * 8;
+            cp_async_16(smem_u32(&sm.k[buf][rr][ch * 8]), p.k + tok * p.k_stride + hd, ok);
+            cp_async_16(smem_u32(&sm.v[buf][rr][ch * 8]), p.v + tok * p.v_stride + hd, ok);
         }
         cp_async_commit();
     };
