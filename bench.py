@@ -336,6 +336,15 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     sh = batch.shape
     bytes_ = algorithmic_bytes(batch)
     q, k, v = batch.q, batch.k, batch.v
+    paged = None
+    if args.page_size:
+        # the same keys in a paged cache: shuffled pages of page_size tokens,
+        # one block-table row per sequence (only step 0's lengths are placed,
+        # so one draw of lengths)
+        if args.workload == "continuous":
+            raise SystemExit("--page-size: the continuous workload changes its lengths every step")
+        paged = W.paginate(k, v, batch.cu_k, sh.B, args.page_size, sh.s_max, seed=0, fill=0.0)
+        k, v = paged.k_cache, paged.v_cache
     cu_q = torch.from_numpy(batch.cu_q).to(dev)
     cu_k = torch.from_numpy(batch.cu_k).to(dev)
     out = torch.empty_like(q)
@@ -369,6 +378,11 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     in0 = torch.cuda.Event(enable_timing=True, external=True)
     in1 = torch.cuda.Event(enable_timing=True, external=True)
 
+    def call(qq, kk, vv, cq, ck, oo, ll):
+        if paged is None:
+            return plan.run(qq, kk, vv, cq, ck, oo, ll)
+        return plan.run_paged(qq, kk, vv, paged.block_table, cq, ck, oo, ll)
+
     def capture(n_calls, events=False):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream, capture_error_mode="global"):
@@ -376,13 +390,13 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
                 in0.record(stream)
             for r in range(n_calls):
                 qq, kk, vv, oo, ll = copies[r]
-                plan.run(qq, kk, vv, cu_q, cu_rows[r], oo, ll)
+                call(qq, kk, vv, cu_q, cu_rows[r], oo, ll)
             if events:
                 in1.record(stream)
         return g
 
     with torch.cuda.stream(stream):
-        plan.run(q, k, v, cu_q, cu_rows[0], out, lse)
+        call(q, k, v, cu_q, cu_rows[0], out, lse)
         stream.synchronize()
         g_iso = capture(1, events=True)
         g_all = capture(n_copies) if pipelined else None
@@ -447,7 +461,8 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     peak, peak_src = measured_peak()
     kernel = {1: "split_simt_kernel", 2: "split_mma_kernel", 3: "split_tc_kernel"}[info["variant"]]
     achieved = timed_bytes / (total_ms * 1e-3) / 1e9
-    traffic, traffic_note = recorded_traffic(args.workload, kernel)
+    traffic_key = args.workload + (f"_paged{args.page_size}" if paged is not None else "")
+    traffic, traffic_note = recorded_traffic(traffic_key, kernel)
     roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": timed_bytes / args.steps,
@@ -461,17 +476,24 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     if not args.no_e2e:
         n_e2e = max(3, min(args.steps, 20))
         # only the tokens this step's lengths cover cross the bus
-        tkv = batch.kv_tokens
+        tkv = batch.kv_tokens if paged is None else k.shape[0]
         hq = batch.q.cpu().pin_memory()
-        hk = batch.k[:tkv].cpu().pin_memory()
-        hv = batch.v[:tkv].cpu().pin_memory()
+        hk = k[:tkv].cpu().pin_memory()
+        hv = v[:tkv].cpu().pin_memory()
         hcq = torch.from_numpy(batch.cu_q).pin_memory()
         hck = torch.from_numpy(batch.cu_k).pin_memory()
         ho = torch.empty_like(hq).pin_memory()
         hl = torch.empty(hq.shape[0], sh.Hq, dtype=torch.float32).pin_memory()
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        if paged is not None:
+            # the halves of one buffer stay views of one buffer
+            dk, dv = torch.empty_like(k.contiguous()), torch.empty_like(v.contiguous())
+            hbt = paged.block_table.cpu().pin_memory()
+            dbt = torch.empty_like(paged.block_table)
         dcq, dck = torch.empty_like(cu_q), torch.empty_like(cu_k)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
+        if paged is not None:
+            h2d += hbt.numel() * hbt.element_size()
         d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
         with torch.cuda.stream(stream):
             def e2e_step():
@@ -480,7 +502,11 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
                 dv[:tkv].copy_(hv, non_blocking=True)
                 dcq.copy_(hcq, non_blocking=True)
                 dck.copy_(hck, non_blocking=True)
-                o, l_ = plan.run(dq, dk, dv, dcq, dck, out, lse)
+                if paged is None:
+                    o, l_ = plan.run(dq, dk, dv, dcq, dck, out, lse)
+                else:
+                    dbt.copy_(hbt, non_blocking=True)
+                    o, l_ = plan.run_paged(dq, dk, dv, dbt, dcq, dck, out, lse)
                 ho.copy_(o, non_blocking=True)
                 hl.copy_(l_, non_blocking=True)
             for _ in range(2):
@@ -509,6 +535,9 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
             "config": {"workload": DESCRIPTIONS[args.workload], "B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv,
                        "D": sh.D, "max_q": sh.max_q, "s_max": sh.s_max,
                        "kv_tokens": int(batch.lens_k.sum()), "q_tokens": int(batch.lens_q.sum()),
+                       "kv_layout": ("packed THD" if paged is None else
+                                     f"paged: {k.shape[0]} pages of {args.page_size} tokens in shuffled "
+                                     f"order, one block-table row per sequence"),
                        "bytes_per_call": timed_bytes / args.steps, "lse_bytes_per_call": bytes_["lse"],
                        "length_draws_cycled": n_var,
                        "l2": (f"inputs larger than L2: {n_copies} copies of the inputs ({n_copies} x "
@@ -551,6 +580,8 @@ def main():
     ap.add_argument("--stages", type=int, default=0)
     ap.add_argument("--combine", type=int, default=0)
     ap.add_argument("--ctas", type=int, default=0)
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="read K/V from a paged cache with pages of this many tokens (0: packed)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()

@@ -64,6 +64,7 @@ extern "C" {
 #define ATTN_DEV_ERR_Q_TOO_LONG 0x2u   /* Lq_b > max_q of the plan            */
 #define ATTN_DEV_ERR_K_TOO_LONG 0x4u   /* Lk_b > s_max of the plan            */
 #define ATTN_DEV_ERR_TIMEOUT 0x8u      /* a bounded pipeline wait gave up      */
+#define ATTN_DEV_ERR_PAGE 0x10u        /* a block-table entry outside the cache */
 
 /* Kernel variants (attn_overrides.variant / attn_plan_desc.variant). */
 #define ATTN_VARIANT_AUTO 0
@@ -208,6 +209,47 @@ int attn_run(attn_plan_t plan, const void *q, const void *k, const void *v,
 int attn_run_strided(attn_plan_t plan, const void *q, const void *k, const void *v,
                      const int32_t *cu_q, const int32_t *cu_k, void *out, float *lse,
                      int64_t k_token_stride, int64_t v_token_stride, void *stream);
+
+/*
+ * attn_run_paged -- attn_run over a paged K/V cache.
+ *
+ *   k_cache, v_cache  device, bf16, 16-byte aligned: num_pages pages of
+ *          page_size tokens, each token Hkv heads of D contiguous elements.
+ *          Token t of page n starts at element n * page_stride +
+ *          t * token_stride of its cache.  K and V share the layout; a cache
+ *          laid out [pages, 2, page_size, Hkv, D] passes v_cache = k_cache +
+ *          page_size * Hkv * D and page_stride = 2 * page_size * Hkv * D.
+ *   page_stride, token_stride  elements; multiples of 8 (16-byte rows),
+ *          token_stride >= Hkv * D, page_stride >= page_size * token_stride,
+ *          both at most 2^38.
+ *   page_size  tokens per page: a power of two, 8 <= page_size <= 2^20.
+ *   num_pages  pages in each cache, >= 1; num_pages * page_size < 2^31.
+ *   block_table  device, int32 [B_max, bt_stride], 4-byte aligned: key j of
+ *          sequence b is token j % page_size of page
+ *          block_table[b * bt_stride + j / page_size].  Only the entries
+ *          covering the sequence's Lk_b keys are read.
+ *   bt_stride  entries per sequence row, >= ceil(s_max / page_size).
+ *   cu_k   as for attn_run, but only the lengths Lk_b = cu_k[b+1] - cu_k[b]
+ *          are used; where the keys sit comes from the block table.
+ *
+ * The keys past Lk_b in a sequence's last page are never used, whatever they
+ * hold (stale or non-finite values included).  A table entry outside
+ * [0, num_pages) sets ATTN_DEV_ERR_PAGE; the keys it names read as zeros, so
+ * the call stays inside the cache, but that sequence's output is then
+ * meaningless.  Bad sizes or strides return ATTN_E_INVALID_ARG and launch
+ * nothing.  Everything else (outputs, capture, error behaviour) is as for
+ * attn_run.  Not available through attn_run_noalloc.
+ *
+ * Source: the paged cache in the split kernel's interface (page size and
+ * page bytes among its parameters), magik.net "Wiring Split-K Dispatch into
+ * a Custom CUDA Attention Kernel", section "The Message: A Read That Reveals
+ * the Architecture"; device-side lengths with the padded positions masked,
+ * TransformerEngine PR #24, section Changes.
+ */
+int attn_run_paged(attn_plan_t plan, const void *q, const void *k_cache, const void *v_cache,
+                   int64_t page_stride, int64_t token_stride, int page_size, int num_pages,
+                   const int32_t *block_table, int bt_stride, const int32_t *cu_q,
+                   const int32_t *cu_k, void *out, float *lse, void *stream);
 
 /*
  * attn_check_error -- synchronise `stream`, then read and clear the plan's

@@ -199,3 +199,35 @@ def merge(o, m, l):
     lse = np.empty((1,), dtype=np.float64)
     lib.oracle_merge(D, S, _ptr(o), _ptr(m), _ptr(l), _ptr(out), _ptr(lse))
     return out, float(lse[0])
+
+
+def gather_pages(cache, block_table, page_size, cu_k, *, B):
+    """Packed [sum Lk_b, Hkv, D] keys (or values) of a paged cache, in key
+    order: key j of sequence b is slot j % page_size of page
+    block_table[b, j // page_size] (the paged cache of the split kernel's
+    interface, magik.net "Wiring Split-K Dispatch into a Custom CUDA Attention
+    Kernel", section "The Message: A Read That Reveals the Architecture").
+    Returns (packed, cu) with cu the prefix sums of the lengths cu_k gives."""
+    cache = _u16(cache, "cache")
+    bt = np.asarray(block_table)
+    cu_k = _i32(cu_k, "cu_k")
+    lens = np.diff(cu_k[: B + 1].astype(np.int64))
+    parts = []
+    for b in range(B):
+        j = np.arange(int(lens[b]))
+        pages = bt[b, j // page_size].astype(np.int64)
+        if pages.size and (pages.min() < 0 or pages.max() >= cache.shape[0]):
+            raise ValueError(f"block table row {b} names a page outside the cache")
+        parts.append(cache[pages, j % page_size])
+    packed = np.concatenate(parts) if parts else cache[:0, 0]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return np.ascontiguousarray(packed), cu
+
+
+def attention_paged(q, k_cache, v_cache, block_table, page_size, cu_q, cu_k, *, B, Hq, Hkv, D, scale=None,
+                    causal=True):
+    """attention() with K and V read from a paged cache ([num_pages,
+    page_size, Hkv, D] uint16 each); only the lengths are taken from cu_k."""
+    k, cu = gather_pages(k_cache, block_table, page_size, cu_k, B=B)
+    v, _ = gather_pages(v_cache, block_table, page_size, cu_k, B=B)
+    return attention(q, k, v, cu_q, cu, B=B, Hq=Hq, Hkv=Hkv, D=D, scale=scale, causal=causal)

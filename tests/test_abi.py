@@ -32,8 +32,8 @@ def libvgqa():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_run_strided", "attn_check_error",
-              "attn_destroy", "attn_strerror", "attn_run_noalloc"):
+    for n in ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_run_strided", "attn_run_paged",
+              "attn_check_error", "attn_destroy", "attn_strerror", "attn_run_noalloc"):
         assert n in names
 
 
@@ -74,6 +74,10 @@ def test_strerror_and_host_errors_without_gpu(libvgqa):
     assert lib.attn_run(None, None, None, None, None, None, None, None, None) == -5
     lib.attn_run_strided.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
     assert lib.attn_run_strided(None, None, None, None, None, None, None, None, 1024, 1024, None) == -5
+    lib.attn_run_paged.argtypes = ([ctypes.c_void_p] * 4 + [ctypes.c_int64] * 2 + [ctypes.c_int] * 2 +
+                                   [ctypes.c_void_p, ctypes.c_int] + [ctypes.c_void_p] * 5)
+    assert lib.attn_run_paged(None, None, None, None, 2048, 256, 16, 4, None, 8, None, None, None, None,
+                              None) == -5
     lib.attn_plan_info.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     buf = ctypes.create_string_buffer(256)
     assert lib.attn_plan_info(ctypes.c_void_p(0x1234), buf) == -5          # unknown handle

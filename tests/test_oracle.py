@@ -495,3 +495,65 @@ def test_longer_cu_buffer_is_zero_length_padding():
         o2, l2 = run(q, k, v, lens, lens, Hq, Hkv, D, B_max=5)
         np.testing.assert_array_equal(np.nan_to_num(o1, nan=3.0), np.nan_to_num(o2, nan=3.0))
         np.testing.assert_array_equal(np.nan_to_num(l1, nan=3.0), np.nan_to_num(l2, nan=3.0))
+
+
+# ------------------------------------------------------------ paged K/V
+
+def _paged_case(page_size, seed, fused=False):
+    sh = W.Shape("paged", B=5, Hq=8, Hkv=2, D=64, max_q=3, s_max=70)
+    batch = W.make_batch(sh, [1, 3, 2, 1, 2], [0, 70, 9, 16, 33], seed=seed)
+    pc = W.paginate(batch.k, batch.v, batch.cu_k, sh.B, page_size, sh.s_max, seed=seed, fused=fused)
+    return sh, batch, pc
+
+
+@pytest.mark.parametrize("page_size", [8, 16, 64])
+def test_gather_pages_follows_the_block_table_by_loops(page_size):
+    """Element by element: key j of sequence b is slot j % page_size of page
+    block_table[b][j // page_size]; the packed offsets are the running sums of
+    the lengths."""
+    sh, batch, pc = _paged_case(page_size, seed=4)
+    kc = W.bits(pc.k_cache)
+    bt = pc.block_table.numpy()
+    packed, cu = oracle.gather_pages(kc, bt, page_size, batch.cu_k, B=sh.B)
+    lens = np.diff(batch.cu_k)
+    assert cu.tolist() == [0] + list(np.cumsum(lens))
+    for b in range(sh.B):
+        for j in range(int(lens[b])):
+            page, slot = int(bt[b][j // page_size]), j % page_size
+            for hk in range(sh.Hkv):
+                for d in range(0, sh.D, 7):
+                    assert packed[cu[b] + j, hk, d] == kc[page, slot, hk, d]
+
+
+@pytest.mark.parametrize("page_size,fused", [(8, False), (16, True), (64, False)])
+def test_paged_attention_equals_packed(page_size, fused):
+    """The same keys reached through a shuffled page table, with every slot no
+    key uses holding NaN, give bit-identical results to the packed layout."""
+    sh, batch, pc = _paged_case(page_size, seed=5, fused=fused)
+    ref_o, ref_l = oracle.attention(W.bits(batch.q), W.bits(batch.k), W.bits(batch.v), batch.cu_q, batch.cu_k,
+                                    B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D)
+    o, l = oracle.attention_paged(W.bits(batch.q), W.bits(pc.k_cache), W.bits(pc.v_cache),
+                                  pc.block_table.numpy(), page_size, batch.cu_q, batch.cu_k, B=sh.B, Hq=sh.Hq,
+                                  Hkv=sh.Hkv, D=sh.D)
+    assert np.array_equal(o, ref_o, equal_nan=True)
+    assert np.array_equal(l, ref_l, equal_nan=True)
+    assert np.all(np.isfinite(o[: int(batch.cu_q[-1])]))
+
+
+def test_paged_attention_ignores_physical_placement():
+    sh, batch, pc1 = _paged_case(16, seed=6)
+    pc2 = W.paginate(batch.k, batch.v, batch.cu_k, sh.B, 16, sh.s_max, seed=99, spare_pages=11)
+    assert not np.array_equal(pc1.block_table.numpy(), pc2.block_table.numpy())
+    res = [oracle.attention_paged(W.bits(batch.q), W.bits(pc.k_cache), W.bits(pc.v_cache),
+                                  pc.block_table.numpy(), 16, batch.cu_q, batch.cu_k, B=sh.B, Hq=sh.Hq,
+                                  Hkv=sh.Hkv, D=sh.D) for pc in (pc1, pc2)]
+    assert np.array_equal(res[0][0], res[1][0], equal_nan=True)
+    assert np.array_equal(res[0][1], res[1][1], equal_nan=True)
+
+
+def test_gather_pages_rejects_a_page_outside_the_cache():
+    sh, batch, pc = _paged_case(16, seed=7)
+    bt = pc.block_table.numpy().copy()
+    bt[1, 2] = pc.k_cache.shape[0]                  # sequence 1 has 70 keys: its third page is used
+    with pytest.raises(ValueError):
+        oracle.gather_pages(W.bits(pc.k_cache), bt, 16, batch.cu_k, B=sh.B)

@@ -24,9 +24,10 @@ ATTN_DEV_ERR_OFFSETS = 0x1
 ATTN_DEV_ERR_Q_TOO_LONG = 0x2
 ATTN_DEV_ERR_K_TOO_LONG = 0x4
 ATTN_DEV_ERR_TIMEOUT = 0x8
+ATTN_DEV_ERR_PAGE = 0x10
 
-EXPORTED = ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_check_error",
-            "attn_destroy", "attn_strerror")
+EXPORTED = ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_run_strided", "attn_run_paged",
+            "attn_check_error", "attn_destroy", "attn_strerror")
 
 
 class Overrides(ctypes.Structure):
@@ -74,6 +75,9 @@ def lib() -> ctypes.CDLL:
         L.attn_run.restype = i
         L.attn_run_strided.argtypes = [vp, vp, vp, vp, i32p, i32p, vp, vp, ctypes.c_int64, ctypes.c_int64, vp]
         L.attn_run_strided.restype = i
+        i64 = ctypes.c_int64
+        L.attn_run_paged.argtypes = [vp, vp, vp, vp, i64, i64, i, i, i32p, i, i32p, i32p, vp, vp, vp]
+        L.attn_run_paged.restype = i
         L.attn_check_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.attn_check_error.restype = i
         L.attn_destroy.argtypes = [vp]
@@ -141,13 +145,8 @@ class Plan:
         fused [T, 2, Hkv, D] cache), which go through attn_run_strided;
         cu_q / cu_k int32 CUDA tensors with B_max + 1 entries; out / lse are
         allocated when not given (pass them for graph capture)."""
-        if self._h is None:
-            raise AttnError(-5, "attn_run")
+        out, lse = self._check_common(q, cu_q, cu_k, out, lse, "attn_run")
         i = self.info
-        if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
-            raise TypeError("q must be a contiguous bf16 CUDA tensor")
-        if q.dim() != 3 or q.shape[1:] != (i["Hq"], i["D"]):
-            raise ValueError(f"q must be [T_q, {i['Hq']}, {i['D']}]")
         for name, t in (("k", k), ("v", v)):
             if t.dtype != torch.bfloat16 or not t.is_cuda:
                 raise TypeError(f"{name} must be a bf16 CUDA tensor")
@@ -155,17 +154,6 @@ class Plan:
                 raise ValueError(f"{name} must be [T_kv, {i['Hkv']}, {i['D']}]")
             if t.stride(2) != 1 or t.stride(1) != i["D"] or (t.shape[0] > 1 and t.stride(0) < i["Hkv"] * i["D"]):
                 raise ValueError(f"{name} must keep each token's heads contiguous (strides (s, D, 1), s >= Hkv*D)")
-        for name, t in (("cu_q", cu_q), ("cu_k", cu_k)):
-            if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.numel() != i["B_max"] + 1:
-                raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of B_max+1 entries")
-        if out is None:
-            out = torch.empty_like(q)
-        if lse is None:
-            lse = torch.empty(q.shape[0], i["Hq"], dtype=torch.float32, device=q.device)
-        if out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous():
-            raise ValueError("out must be a contiguous bf16 tensor shaped like q")
-        if lse.dtype != torch.float32 or lse.shape != (q.shape[0], i["Hq"]) or not lse.is_contiguous():
-            raise ValueError("lse must be a contiguous fp32 tensor [T_q, Hq]")
         packed = i["Hkv"] * i["D"]
         ks = k.stride(0) if k.shape[0] > 1 else packed
         vs = v.stride(0) if v.shape[0] > 1 else packed
@@ -178,6 +166,65 @@ class Plan:
                                         cu_k.data_ptr(), out.data_ptr(), lse.data_ptr(), ks, vs,
                                         _stream_ptr(stream))
             _check(rc, "attn_run_strided")
+        return out, lse
+
+    def run_paged(self, q, k_cache, v_cache, block_table, cu_q, cu_k, out=None, lse=None, stream=None):
+        """out, lse = plan.run_paged(q, k_cache, v_cache, block_table, cu_q, cu_k[, out, lse, stream]).
+
+        k_cache / v_cache [num_pages, page_size, Hkv, D] bf16 CUDA tensors
+        (each token's heads contiguous; token and page strides free, so the
+        halves of a [num_pages, 2, page_size, Hkv, D] cache work);
+        block_table [B_max, n] int32 CUDA tensor, row b listing the pages of
+        sequence b in key order (n >= ceil(s_max / page_size), row stride
+        free); cu_k supplies the key lengths only.  Goes through
+        attn_run_paged."""
+        out, lse = self._check_common(q, cu_q, cu_k, out, lse, "attn_run_paged")
+        i = self.info
+        shape = None
+        for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+            if t.dtype != torch.bfloat16 or not t.is_cuda:
+                raise TypeError(f"{name} must be a bf16 CUDA tensor")
+            if t.dim() != 4 or t.shape[2:] != (i["Hkv"], i["D"]):
+                raise ValueError(f"{name} must be [num_pages, page_size, {i['Hkv']}, {i['D']}]")
+            if t.stride(3) != 1 or t.stride(2) != i["D"]:
+                raise ValueError(f"{name} must keep each token's heads contiguous")
+            if shape is not None and (t.shape != shape or t.stride() != k_cache.stride()):
+                raise ValueError("k_cache and v_cache must have the same shape and strides")
+            shape = t.shape
+        n_pages, page_size = int(shape[0]), int(shape[1])
+        tok = k_cache.stride(1) if page_size > 1 else i["Hkv"] * i["D"]
+        pstride = k_cache.stride(0) if n_pages > 1 else page_size * tok
+        bt = block_table
+        if bt.dtype != torch.int32 or not bt.is_cuda or bt.dim() != 2 or bt.shape[0] != i["B_max"] or bt.stride(1) != 1:
+            raise ValueError("block_table must be an int32 CUDA tensor [B_max, n] with unit column stride")
+        if bt.shape[1] * page_size < i["s_max"]:
+            raise ValueError("block_table rows must cover s_max keys")
+        rc = lib().attn_run_paged(self._h, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), int(pstride),
+                                  int(tok), page_size, n_pages, bt.data_ptr(), int(bt.stride(0)),
+                                  cu_q.data_ptr(), cu_k.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  _stream_ptr(stream))
+        _check(rc, "attn_run_paged")
+        return out, lse
+
+    def _check_common(self, q, cu_q, cu_k, out, lse, where):
+        if self._h is None:
+            raise AttnError(-5, where)
+        i = self.info
+        if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
+            raise TypeError("q must be a contiguous bf16 CUDA tensor")
+        if q.dim() != 3 or q.shape[1:] != (i["Hq"], i["D"]):
+            raise ValueError(f"q must be [T_q, {i['Hq']}, {i['D']}]")
+        for name, t in (("cu_q", cu_q), ("cu_k", cu_k)):
+            if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.numel() != i["B_max"] + 1:
+                raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of B_max+1 entries")
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(q.shape[0], i["Hq"], dtype=torch.float32, device=q.device)
+        if out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous():
+            raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+        if lse.dtype != torch.float32 or lse.shape != (q.shape[0], i["Hq"]) or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous fp32 tensor [T_q, Hq]")
         return out, lse
 
     def check_error(self, stream=None) -> int:

@@ -62,15 +62,35 @@ int get_encoder() {
 }
 
 // [T, Hkv, D] bf16, box = 64 elements x 1 head x block_n tokens, 128-byte
-// swizzle.  The token extent is left open (2^31 - 1): every load the kernel
-// issues ends at or before its sequence's last key (cu_k[b+1] - 1), so the
-// real buffer length never enters.
-int encode_kv_map(CUtensorMap *map, const void *base, int Hkv, int D, int block_n, long long token_stride) {
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)0x7fffffff};
+// swizzle.  Packed K/V leave the token extent open (2^31 - 1): every load the
+// kernel issues ends at or before its sequence's last key (cu_k[b+1] - 1), so
+// the real buffer length never enters.  A paged cache passes its row count,
+// so a load at row num_pages * page_rows (the kernels' stand-in for a key
+// past the sequence or a bad table entry) lies outside and fills zeros.
+int encode_kv_map(CUtensorMap *map, const void *base, int Hkv, int D, int block_n, long long token_stride,
+                  long long rows = 0x7fffffff) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)token_stride * 2};
     cuuint32_t box[3] = {64, 1, (cuuint32_t)block_n};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
+}
+
+// Paged cache [pages, page_size, Hkv, D] bf16 with explicit token and page
+// strides, box = 64 elements x 1 head x min(page_size, 64) tokens x 1 page,
+// 128-byte swizzle.  A load at page index num_pages (the kernels' stand-in
+// for a key past the sequence or a bad table entry) lies wholly outside the
+// map and is filled with zeros.
+int encode_paged_map(CUtensorMap *map, const void *base, int Hkv, int D, int page_size, int num_pages,
+                     long long token_stride, long long page_stride) {
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)page_size, (cuuint64_t)num_pages};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)token_stride * 2, (cuuint64_t)page_stride * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)std::min(page_size, 64), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
@@ -327,8 +347,22 @@ ATTN_EXPORT int attn_plan_info(attn_plan_t plan, attn_plan_desc *desc) {
 
 namespace {
 
+// where the keys live when the cache is paged (attn_run_paged)
+struct Paging {
+    const int32_t *block_table;
+    int bt_stride, page_size, num_pages;
+    long long page_stride;
+};
+
+int log2_exact(long long x) {
+    int s = 0;
+    while ((1ll << s) < x) ++s;
+    return (1ll << s) == x ? s : -1;
+}
+
 int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, const int32_t *cu_q,
-             const int32_t *cu_k, void *out, float *lse, long long k_stride, long long v_stride, void *stream) {
+             const int32_t *cu_k, void *out, float *lse, long long k_stride, long long v_stride,
+             const Paging *pg, void *stream) {
     if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
     if (!q || !k || !v || !cu_q || !cu_k || !out || !lse) return ATTN_E_NULL;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
@@ -364,6 +398,18 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     p.scale_log2 = plan->scale_log2;
     p.k_stride = k_stride;
     p.v_stride = v_stride;
+    if (pg) {
+        p.block_table = pg->block_table;
+        p.bt_stride = pg->bt_stride;
+        p.page_shift = log2_exact(pg->page_size);
+        p.num_pages = pg->num_pages;
+        p.page_box = std::min(pg->page_size, 64);
+        p.page_stride = pg->page_stride;
+        // pages a whole number of token rows apart: one row index per key,
+        // page * page_rows + slot, into a 3-D map of all the cache's rows
+        if (pg->page_stride % k_stride == 0 && (long long)pg->num_pages * (pg->page_stride / k_stride) < (1ll << 31))
+            p.page_rows = (int)(pg->page_stride / k_stride);
+    }
     p.ticket = plan->ticket;
     p.claim = reinterpret_cast<unsigned long long *>(plan->ticket);
     p.done = plan->ticket + 2 * (size_t)d.B_max * d.Hkv;
@@ -377,18 +423,30 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(d.grid_x, d.grid_y, d.grid_z);
+    // K and V tensor maps of the TMA-fed kernels
+    auto kv_maps = [&](CUtensorMap &tm_k, CUtensorMap &tm_v) -> bool {
+        if (pg && p.page_rows) {
+            const long long rows = (long long)pg->num_pages * p.page_rows;
+            const int box = std::min(pg->page_size, 64);
+            return encode_kv_map(&tm_k, k, d.Hkv, d.D, box, k_stride, rows) == ATTN_OK &&
+                   encode_kv_map(&tm_v, v, d.Hkv, d.D, box, v_stride, rows) == ATTN_OK;
+        }
+        if (pg)
+            return encode_paged_map(&tm_k, k, d.Hkv, d.D, pg->page_size, pg->num_pages, k_stride,
+                                    pg->page_stride) == ATTN_OK &&
+                   encode_paged_map(&tm_v, v, d.Hkv, d.D, pg->page_size, pg->num_pages, v_stride,
+                                    pg->page_stride) == ATTN_OK;
+        return encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n, k_stride) == ATTN_OK &&
+               encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n, v_stride) == ATTN_OK;
+    };
     cudaError_t e;
     if (d.variant == ATTN_VARIANT_MMA) {
         CUtensorMap tm_k, tm_v;
-        if (encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n, k_stride) != ATTN_OK ||
-            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n, v_stride) != ATTN_OK)
-            return ATTN_E_CUDA;
+        if (!kv_maps(tm_k, tm_v)) return ATTN_E_CUDA;
         e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, d.ctas, s);
     } else if (d.variant == ATTN_VARIANT_TC) {
         CUtensorMap tm_q, tm_k, tm_v;
-        if (encode_q_map(&tm_q, q, d.Hq, d.D, d.G, d.max_q) != ATTN_OK ||
-            encode_kv_map(&tm_k, k, d.Hkv, d.D, d.block_n, k_stride) != ATTN_OK ||
-            encode_kv_map(&tm_v, v, d.Hkv, d.D, d.block_n, v_stride) != ATTN_OK)
+        if (encode_q_map(&tm_q, q, d.Hq, d.D, d.G, d.max_q) != ATTN_OK || !kv_maps(tm_k, tm_v))
             return ATTN_E_CUDA;
         e = launch_split_tc(p, tm_q, tm_k, tm_v, d.stages, d.ctas, s);
     } else {
@@ -408,7 +466,7 @@ ATTN_EXPORT int attn_run(attn_plan_t plan, const void *q, const void *k, const v
                          const int32_t *cu_k, void *out, float *lse, void *stream) {
     if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
     const long long packed = (long long)plan->d.Hkv * plan->d.D;
-    return run_impl(plan, q, k, v, cu_q, cu_k, out, lse, packed, packed, stream);
+    return run_impl(plan, q, k, v, cu_q, cu_k, out, lse, packed, packed, nullptr, stream);
 }
 
 ATTN_EXPORT int attn_run_strided(attn_plan_t plan, const void *q, const void *k, const void *v,
@@ -420,7 +478,31 @@ ATTN_EXPORT int attn_run_strided(attn_plan_t plan, const void *q, const void *k,
     // alignment (the tensor-map rule) and fits the tensor map's range
     for (long long st : {(long long)k_token_stride, (long long)v_token_stride})
         if (st < packed || st % 8 != 0 || st > (1ll << 38)) return ATTN_E_INVALID_ARG;
-    return run_impl(plan, q, k, v, cu_q, cu_k, out, lse, k_token_stride, v_token_stride, stream);
+    return run_impl(plan, q, k, v, cu_q, cu_k, out, lse, k_token_stride, v_token_stride, nullptr, stream);
+}
+
+ATTN_EXPORT int attn_run_paged(attn_plan_t plan, const void *q, const void *k_cache, const void *v_cache,
+                               int64_t page_stride, int64_t token_stride, int page_size, int num_pages,
+                               const int32_t *block_table, int bt_stride, const int32_t *cu_q,
+                               const int32_t *cu_k, void *out, float *lse, void *stream) {
+    if (!plan || !live(plan)) return ATTN_E_BAD_PLAN;
+    if (!block_table) return ATTN_E_NULL;
+    if (!aligned(block_table, 4)) return ATTN_E_ALIGNMENT;
+    const attn_plan_desc &d = plan->d;
+    const long long packed = (long long)d.Hkv * d.D;
+    // power-of-two pages of at least 8 tokens: a tile of 64 keys then covers
+    // whole pages or lies inside one, and each TMA box starts on a 1 KB
+    // boundary of the 128-byte swizzle pattern
+    const int shift = log2_exact(page_size);
+    if (page_size < 8 || page_size > (1 << 20) || shift < 0 || num_pages < 1 ||
+        (long long)num_pages * page_size >= (1ll << 31))
+        return ATTN_E_INVALID_ARG;
+    if (token_stride < packed || token_stride % 8 != 0 || token_stride > (1ll << 38) || page_stride % 8 != 0 ||
+        page_stride < (long long)page_size * token_stride || page_stride > (1ll << 38))
+        return ATTN_E_INVALID_ARG;
+    if (bt_stride < (d.s_max + page_size - 1) / page_size) return ATTN_E_INVALID_ARG;
+    const Paging pg{block_table, bt_stride, page_size, num_pages, page_stride};
+    return run_impl(plan, q, k_cache, v_cache, cu_q, cu_k, out, lse, token_stride, token_stride, &pg, stream);
 }
 
 ATTN_EXPORT int attn_check_error(attn_plan_t plan, void *stream, uint32_t *flags) {

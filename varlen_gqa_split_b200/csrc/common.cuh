@@ -56,6 +56,40 @@ __device__ __forceinline__ bool load_lengths(const Params &p, int b, bool report
     return bad == 0;
 }
 
+// Paged K/V: the page holding key j of sequence b, from the block table, in
+// two steps so that the table read can overlap a wait: page_entry() issues
+// the read, page_checked() validates the value.  An entry outside
+// [0, num_pages) raises ATTN_DEV_ERR_PAGE and gives num_pages, a page past
+// the cache: tensor-map loads of it fill zeros and the CUDA-core path skips
+// it, so a bad table never reads outside the cache.
+__device__ __forceinline__ int page_entry(const Params &p, int b, int j) {
+    // volatile: stays ahead of the (volatile) barrier wait that follows it,
+    // so the read is in flight during the wait
+    int pg;
+    asm volatile("ld.global.nc.b32 %0, [%1];"
+                 : "=r"(pg)
+                 : "l"(p.block_table + (long long)b * p.bt_stride + (j >> p.page_shift)));
+    return pg;
+}
+__device__ __forceinline__ int page_checked(const Params &p, int pg) {
+    if ((unsigned)pg >= (unsigned)p.num_pages) {
+        atomicOr(p.err, ATTN_DEV_ERR_PAGE);
+        return p.num_pages;
+    }
+    return pg;
+}
+__device__ __forceinline__ int page_of(const Params &p, int b, int j) { return page_checked(p, page_entry(p, b, j)); }
+
+// pull the block-table entries of keys [0, Lk) of sequence b into L2 (one
+// prefetch per 128-byte line), so the per-tile reads that follow hit there
+__device__ __forceinline__ void prefetch_pages(const Params &p, int b, int Lk) {
+    const int32_t *row = p.block_table + (long long)b * p.bt_stride;
+    const int n = (Lk + (1 << p.page_shift) - 1) >> p.page_shift;
+    for (int i = 0; i < n; i += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + i));
+}
+
+constexpr int kMaxPageBoxes = 8;          // paged K/V: boxes per 64-key tile at the smallest page (8 keys)
+
 // ------------------------------------------------------------ small math
 
 __device__ __forceinline__ float ex2(float x) {   // SFU exp2 (ex2(-inf) = +0)
@@ -138,6 +172,16 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+        "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, int c2, int c3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
         "l"(policy)
         : "memory");
 }

@@ -36,6 +36,16 @@ struct Params {
     int share_stride;          // tensor-core path: block b takes share (b * share_stride) mod blocks
     long long k_stride;        // elements between consecutive tokens of k (Hkv * D when packed)
     long long v_stride;        // elements between consecutive tokens of v
+    // paged K/V (block_table != null): key j of sequence b sits in page
+    // block_table[b * bt_stride + (j >> page_shift)], slot j & (page size - 1)
+    const int32_t *block_table;
+    int bt_stride;             // entries per sequence row of block_table
+    int page_shift;            // log2(page size)
+    int num_pages;             // pages in the cache (valid page indexes)
+    int page_box;              // keys per TMA load: min(page size, 64)
+    long long page_stride;     // elements between consecutive pages of k and v
+    int page_rows;             // page_stride / token stride when whole (tensor maps index rows
+                               // page * page_rows + slot), else 0 (tensor maps index (slot, page))
 };
 
 }  // namespace vgqa

@@ -247,7 +247,9 @@ __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int t
 // whose static part is the unit's front claims upward, the others downward,
 // kClaim tiles at a time with one claim in flight ahead of the tiles it feeds;
 // each claim gets the part of its range that the counter's old value shows as
-// still free.  A callback returns false to stop the walk (a wait gave up);
+// still free.  A block's claimed tiles of a cut unit all go out with `last`
+// false, followed by none(seg): consumers finish their part of the unit at
+// that empty stage.  A callback returns false to stop the walk (a wait gave up);
 // the function then returns false.
 template <class Begin, class Tile, class None>
 __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long long pb_first, long long lo,
@@ -280,26 +282,23 @@ __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long lo
                 t_lo = max(free_hi - kClaim, f);
             }
         };
-        int a_lo, a_hi, n_lo, n_hi;
+        // The next claim goes out when a range starts and is resolved only
+        // after that range's tiles have been fed, so the atomic's round trip
+        // overlaps them; the tiles therefore cannot be told which one ends
+        // the block's part, and an empty terminator stage (none) marks the
+        // end instead.
+        int a_lo, a_hi;
         range(atomicAdd(claim, inc), a_lo, a_hi);
-        bool any = false;
         while (a_lo < a_hi) {
-            // next claim in flight, unless this one already reached the far end
-            const bool more = up ? a_hi < ntiles : a_lo > 0;
-            if (more)
-                range(atomicAdd(claim, inc), n_lo, n_hi);
-            else
-                n_lo = n_hi = 0;
-            const bool final_range = !(n_lo < n_hi);
-            for (int i = 0; i < a_hi - a_lo; ++i) {
-                const int t = up ? a_lo + i : a_hi - 1 - i;
-                if (!tile(seg, t, final_range && i == a_hi - a_lo - 1)) return false;
-                any = true;
-            }
-            a_lo = n_lo;
-            a_hi = n_hi;
+            const bool more = up ? a_hi < ntiles : a_lo > 0;   // this range did not reach the far end
+            unsigned long long pend = 0;
+            if (more) pend = atomicAdd(claim, inc);
+            for (int i = 0; i < a_hi - a_lo; ++i)
+                if (!tile(seg, up ? a_lo + i : a_hi - 1 - i, false)) return false;
+            if (!more) break;
+            range(pend, a_lo, a_hi);
         }
-        if (!any && !none(seg)) return false;
+        if (!none(seg)) return false;
     }
     return true;
 }

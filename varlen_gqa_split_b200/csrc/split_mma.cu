@@ -144,8 +144,71 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 }
             };
             auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
-                if (!acquire()) return false;
                 const int ks = tile * kBN;
+                if (p.block_table && p.page_box == kBN && p.page_rows) {
+                    // paged, pages of 64 keys or more a whole number of rows apart: one
+                    // row index per tile, page * page_rows + slot, as lean as a packed
+                    // tile (the table read is issued before the stage wait)
+                    const int entry = page_entry(p, sg.b, ks);
+                    if (!acquire()) return false;
+                    const int row = page_checked(p, entry) * p.page_rows + (ks & ((1 << p.page_shift) - 1));
+                    meta[s] = make_int2(ks, last ? kMetaLast : 0);
+                    uint8_t *st = ring + s * L::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+#pragma unroll
+                    for (int hf = 0; hf < L::kHalves; ++hf)
+                        tma_load_3d(st + hf * L::kRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
+#pragma unroll
+                    for (int hf = 0; hf < L::kHalves; ++hf)
+                        tma_load_3d(st + L::kTileBytes + hf * L::kRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
+                    advance();
+                    return true;
+                }
+                if (p.block_table) {
+                    // paged, in general: the tile's keys in boxes of page_box keys,
+                    // each from its page; the table is read before the stage wait,
+                    // so the read overlaps it
+                    const int nbox = kBN / p.page_box;
+                    int pg[kMaxPageBoxes];
+                    uint32_t live = 0;                      // boxes holding keys of the sequence
+#pragma unroll
+                    for (int i = 0; i < kMaxPageBoxes; ++i) {
+                        if (i >= nbox) break;
+                        const int key = ks + i * p.page_box;
+                        pg[i] = 0;
+                        if (key < sg.s.Lk) {
+                            pg[i] = page_entry(p, sg.b, key);
+                            live |= 1u << i;
+                        }
+                    }
+                    if (!acquire()) return false;
+                    meta[s] = make_int2(ks, last ? kMetaLast : 0);
+                    uint8_t *st = ring + s * L::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+                    const int slot_mask = (1 << p.page_shift) - 1;
+#pragma unroll
+                    for (int i = 0; i < kMaxPageBoxes; ++i) {
+                        if (i >= nbox) break;
+                        // a box past the sequence (or a bad entry) reads page num_pages,
+                        // outside the map: zeros
+                        const int page = (live >> i) & 1u ? page_checked(p, pg[i]) : p.num_pages;
+                        const int slot = (ks + i * p.page_box) & slot_mask;   // 0 when pages are < 64 keys
+#pragma unroll
+                        for (int hf = 0; hf < L::kHalves; ++hf) {
+                            uint8_t *dk = st + hf * L::kRegion + i * p.page_box * 128, *dv = dk + L::kTileBytes;
+                            if (p.page_rows) {
+                                tma_load_3d(dk, &tm_k, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
+                                tma_load_3d(dv, &tm_v, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
+                            } else {
+                                tma_load_4d(dk, &tm_k, &full[s], hf * 64, sg.hk, slot, page, pol);
+                                tma_load_4d(dv, &tm_v, &full[s], hf * 64, sg.hk, slot, page, pol);
+                            }
+                        }
+                    }
+                    advance();
+                    return true;
+                }
+                if (!acquire()) return false;
                 const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
                 meta[s] = make_int2(ks, last ? kMetaLast : 0);
                 uint8_t *st = ring + s * L::kStageBytes;
@@ -166,8 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 advance();
                 return true;
             };
-            feed_tiles(p, b_first, pb_first, lo, hi, [](const Segment &, int) { return true; }, load_tile,
-                       empty_stage);
+            auto begin = [&](const Segment &sg, int) -> bool {
+                if (p.block_table) prefetch_pages(p, sg.b, sg.s.Lk);
+                return true;
+            };
+            feed_tiles(p, b_first, pb_first, lo, hi, begin, load_tile, empty_stage);
         }
         return;
     }
@@ -256,7 +322,25 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             const int t0 = mt.x;
             const uint32_t kst = ring_base + s * L::kStageBytes;
             const uint32_t vst = kst + L::kTileBytes;
-            const int ls = min(t0, Lk - kBN);     // key index of tile row 0
+            // key index of tile row 0: a packed tile past the sequence's end
+            // was moved back to end at its last key; a paged tile starts at
+            // t0, and its rows past Lk hold whatever the page held
+            const bool paged = p.block_table != nullptr;
+            const int ls = paged ? t0 : min(t0, Lk - kBN);
+            bool zeroed = false;
+            if (paged && t0 + kBN > Lk) {
+                // zero this warp's V rows past Lk: their weights are 0, but
+                // 0 times a stale non-finite value would not be
+                const int z0 = max(kbase, Lk - t0);
+                uint8_t *vt = ring + s * L::kStageBytes + L::kTileBytes;
+                for (int i = lane; i < (kbase + 16 - z0) * L::kHalves * 8; i += 32) {
+                    const int r = z0 + i / (L::kHalves * 8), rest = i % (L::kHalves * 8);
+                    *reinterpret_cast<uint4 *>(vt + (rest >> 3) * L::kRegion + r * 128 + (rest & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                zeroed = true;
+                __syncwarp();
+            }
 
             // S^T = K Q^T
             float sacc[NT][4];
@@ -314,6 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
             }
 
+            // the generic-proxy zeroing precedes the stage's next TMA write
+            if (zeroed) fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
             if (++s == stages) {

@@ -88,11 +88,19 @@ __global__ void __launch_bounds__(kThreads) split_simt_kernel(const Params p) {
         for (int c = tid; c < kBN * kChunks; c += kThreads) {
             const int rr = c / kChunks, ch = c % kChunks;
             const int j = t0 + rr;
-            const bool ok = j < kv_lim;
-            const long long tok = ok ? (long long)(k0 + j) : 0;
+            bool ok = j < kv_lim;
+            long long ko = 0, vo = 0;                  // element offsets of the key's token
+            if (ok && p.block_table) {                 // paged: page from the block table
+                const int pg = page_of(p, b, j);
+                ok = pg < p.num_pages;
+                ko = vo = (long long)pg * p.page_stride + (long long)(j & ((1 << p.page_shift) - 1)) * p.k_stride;
+            } else if (ok) {
+                ko = (long long)(k0 + j) * p.k_stride;
+                vo = (long long)(k0 + j) * p.v_stride;
+            }
             const long long hd = (long long)hk * D + ch * 8;
-            cp_async_16(smem_u32(&sm.k[buf][rr][ch * 8]), p.k + tok * p.k_stride + hd, ok);
-            cp_async_16(smem_u32(&sm.v[buf][rr][ch * 8]), p.v + tok * p.v_stride + hd, ok);
+            cp_async_16(smem_u32(&sm.k[buf][rr][ch * 8]), p.k + (ok ? ko + hd : 0), ok);
+            cp_async_16(smem_u32(&sm.v[buf][rr][ch * 8]), p.v + (ok ? vo + hd : 0), ok);
         }
         cp_async_commit();
     };

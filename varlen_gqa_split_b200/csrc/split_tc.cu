@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             }
         };
         auto begin = [&](const Segment &sg, int) -> bool {
+            if (p.block_table) prefetch_pages(p, sg.b, sg.s.Lk);
             const int qb = k & 1;
             if (k >= 2 && !wait_bar(&q_free[qb], ((k - 2) >> 1) & 1, stop, p)) return false;
             mbar_arrive_expect_tx(&q_full[qb], q_bytes);
@@ -201,8 +202,71 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             return true;
         };
         auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
-            if (!acquire()) return false;
             const int ks = tile * kBN;
+            if (p.block_table && p.page_box == kBN && p.page_rows) {
+                // paged, pages of 64 keys or more a whole number of rows apart: one
+                // row index per tile, page * page_rows + slot, as lean as a packed
+                // tile (the table read is issued before the stage wait)
+                const int entry = page_entry(p, sg.b, ks);
+                if (!acquire()) return false;
+                const int row = page_checked(p, entry) * p.page_rows + (ks & ((1 << p.page_shift) - 1));
+                meta[s] = make_int2(ks, last ? kMetaLast : 0);
+                uint8_t *st = ring + s * L::kStage;
+                mbar_arrive_expect_tx(&full[s], L::kStage);
+#pragma unroll
+                for (int hf = 0; hf < L::kHalves; ++hf)
+                    tma_load_3d(st + hf * L::kKvRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
+#pragma unroll
+                for (int hf = 0; hf < L::kHalves; ++hf)
+                    tma_load_3d(st + L::kKvTile + hf * L::kKvRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
+                advance();
+                return true;
+            }
+            if (p.block_table) {
+                // paged, in general: the tile's keys in boxes of page_box keys,
+                // each from its page; the table is read before the stage wait,
+                // so the read overlaps it
+                const int nbox = kBN / p.page_box;
+                int pg[kMaxPageBoxes];
+                uint32_t live = 0;                      // boxes holding keys of the sequence
+#pragma unroll
+                for (int i = 0; i < kMaxPageBoxes; ++i) {
+                    if (i >= nbox) break;
+                    const int key = ks + i * p.page_box;
+                    pg[i] = 0;
+                    if (key < sg.s.Lk) {
+                        pg[i] = page_entry(p, sg.b, key);
+                        live |= 1u << i;
+                    }
+                }
+                if (!acquire()) return false;
+                meta[s] = make_int2(ks, last ? kMetaLast : 0);
+                uint8_t *st = ring + s * L::kStage;
+                mbar_arrive_expect_tx(&full[s], L::kStage);
+                const int slot_mask = (1 << p.page_shift) - 1;
+#pragma unroll
+                for (int i = 0; i < kMaxPageBoxes; ++i) {
+                    if (i >= nbox) break;
+                    // a box past the sequence (or a bad entry) reads page num_pages,
+                    // outside the map: zeros
+                    const int page = (live >> i) & 1u ? page_checked(p, pg[i]) : p.num_pages;
+                    const int slot = (ks + i * p.page_box) & slot_mask;   // 0 when pages are < 64 keys
+#pragma unroll
+                    for (int hf = 0; hf < L::kHalves; ++hf) {
+                        uint8_t *dk = st + hf * L::kKvRegion + i * p.page_box * 128, *dv = dk + L::kKvTile;
+                        if (p.page_rows) {
+                            tma_load_3d(dk, &tm_k, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
+                            tma_load_3d(dv, &tm_v, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
+                        } else {
+                            tma_load_4d(dk, &tm_k, &full[s], hf * 64, sg.hk, slot, page, pol);
+                            tma_load_4d(dv, &tm_v, &full[s], hf * 64, sg.hk, slot, page, pol);
+                        }
+                    }
+                }
+                advance();
+                return true;
+            }
+            if (!acquire()) return false;
             const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
             meta[s] = make_int2(ks, last ? kMetaLast : 0);
             uint8_t *st = ring + s * L::kStage;
@@ -284,9 +348,18 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                         s = 0;
                         sph ^= 1;
                     }
-                    if (mt.y & kMetaEmpty) {            // the unit ends without a tile here
+                    if (mt.y & kMetaEmpty) {
+                        // the block's part of the unit ends here: flush the
+                        // deferred product of its last tile, if any, and
+                        // free the Q buffer once the products reading it are
+                        // done (the commit tracks them)
                         mbar_arrive(&empty[cs_]);
-                        mbar_arrive(&q_free[qb]);
+                        if (have_prev) {
+                            if (!(ok = issue_pv())) break;
+                            have_prev = false;
+                            ++e;
+                        }
+                        tc::commit(smem_u32(&q_free[qb]));
                         break;
                     }
                     const int b = j & 1;
@@ -365,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             while (true) {
                 if (!(ok = wwait(&full[s], sph))) break;
                 const int2 mt = meta[s];
+                const int ts = s;                                // this tile's stage
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
                 if (++s == stages) {
@@ -373,6 +447,20 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 }
                 if (mt.y & kMetaEmpty) break;
                 has_tiles = true;
+                if (p.block_table && mt.x + kBN > Lk) {
+                    // paged tile past the sequence's end: zero its V rows
+                    // past Lk (weight 0 times a stale non-finite value would
+                    // not be 0) before this warp's P is signalled; the stage
+                    // is refilled only after the product that follows
+                    const int z0 = Lk - mt.x;
+                    uint8_t *vt = ring + ts * L::kStage + L::kKvTile;
+                    for (int i = tid; i < (kBN - z0) * L::kHalves * 8; i += kSoftWarps * 32) {
+                        const int rr = z0 + i / (L::kHalves * 8), rest = i % (L::kHalves * 8);
+                        *reinterpret_cast<uint4 *>(vt + (rest >> 3) * L::kKvRegion + rr * 128 + (rest & 7) * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async();                         // before the tensor core reads V
+                }
                 const int b = j & 1;
                 if (!(ok = wwait(&s_full[b], (j >> 1) & 1))) break;
                 if (!act) {
@@ -397,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 // mask and max of this half.  The scale (> 0) enters in the
                 // exp2 argument, so the raw maximum gives the scaled one; a
                 // masked score becomes -inf, whose weight is exactly 0.
-                const int ks = mt.x, ls = min(ks, Lk - kBN);     // key of column 0
+                const int ks = mt.x, ls = p.block_table ? ks : min(ks, Lk - kBN);   // key of column 0
                 const int c0 = half * kHalfKeys;
                 const int lo_c = ks - ls - c0, hi_c = min(kHalfKeys, vis - ls - c0);   // visible [lo_c, hi_c)
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};

@@ -198,3 +198,63 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     only."""
     f = np.asarray(x, dtype=np.float32)
     return bits(torch.from_numpy(np.ascontiguousarray(f)).to(torch.bfloat16))
+
+
+# ------------------------------------------------------------ paged K/V caches
+
+@dataclasses.dataclass
+class PagedCache:
+    """A batch's keys and values scattered into a paged cache.
+
+    k_cache / v_cache: [num_pages, page_size, Hkv, D] (views of one
+    [num_pages, 2, page_size, Hkv, D] buffer when fused); block_table:
+    [B_max, cols] int32, row b listing sequence b's pages in key order, every
+    entry past the sequence's pages set to `unused`."""
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_table: torch.Tensor
+    page_size: int
+
+
+def paginate(k: torch.Tensor, v: torch.Tensor, cu_k, B_max: int, page_size: int, s_max: int, *,
+             seed: int = 0, spare_pages: int = 3, fill: float = float("nan"), fused: bool = False,
+             extra_cols: int = 0, unused: int = -7) -> PagedCache:
+    """Place key j of sequence b (packed token cu_k[b] + j) at slot j % page_size
+    of a randomly chosen distinct page; slots no key uses hold `fill` (NaN by
+    default, so a kernel that lets them into its result fails loudly).
+    `spare_pages` pages belong to no sequence."""
+    cu_k = np.asarray(cu_k, dtype=np.int64)
+    lens = np.diff(cu_k[: B_max + 1])
+    Hkv, D = k.shape[1], k.shape[2]
+    n_pages_b = (lens + page_size - 1) // page_size
+    total = int(n_pages_b.sum()) + spare_pages
+    rng = np.random.default_rng(seed)
+    phys = rng.permutation(total)                  # logical page -> physical page
+    cols = (s_max + page_size - 1) // page_size + extra_cols
+    bt = np.full((B_max, cols), unused, dtype=np.int32)
+    first = np.concatenate([[0], np.cumsum(n_pages_b)])
+    rows = []                                       # physical row of each packed key
+    for b in range(B_max):
+        n = int(n_pages_b[b])
+        bt[b, :n] = phys[first[b]: first[b] + n]
+        j = np.arange(int(lens[b]))
+        rows.append(phys[first[b] + j // page_size] * page_size + j % page_size)
+    rows = np.concatenate(rows) if rows else np.zeros(0, np.int64)
+    dev = k.device
+    if fused:
+        buf = torch.full((total, 2, page_size, Hkv, D), fill, dtype=torch.bfloat16, device=dev)
+        kc, vc = buf[:, 0], buf[:, 1]
+    else:
+        kc = torch.full((total, page_size, Hkv, D), fill, dtype=torch.bfloat16, device=dev)
+        vc = torch.full((total, page_size, Hkv, D), fill, dtype=torch.bfloat16, device=dev)
+    idx = torch.from_numpy(rows).to(dev)
+    src = slice(int(cu_k[0]), int(cu_k[0]) + len(rows))
+    # scatter through a flat [pages * page_size, Hkv, D] view of each cache
+    for cache, data in ((kc, k), (vc, v)):
+        flat = cache.reshape(total * page_size, Hkv, D) if cache.is_contiguous() else None
+        if flat is not None:
+            flat[idx] = data[src]
+        else:
+            pg, sl = idx // page_size, idx % page_size
+            cache[pg, sl] = data[src]
+    return PagedCache(kc, vc, torch.from_numpy(bt).to(dev), page_size)
