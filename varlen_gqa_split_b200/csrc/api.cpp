@@ -420,6 +420,7 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     const bool persistent = d.variant == ATTN_VARIANT_MMA || d.variant == ATTN_VARIANT_TC;
     p.dynamic = persistent && !d.deterministic;
     p.done_per_part = d.variant == ATTN_VARIANT_TC ? tc_parts_per_block() : 1;
+    p.unit_cost = d.variant == ATTN_VARIANT_TC ? tc_unit_cost() : 0;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(d.grid_x, d.grid_y, d.grid_z);

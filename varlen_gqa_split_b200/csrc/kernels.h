@@ -35,6 +35,7 @@ size_t tc_smem_need(int D, int stages);    // bytes the layout uses
 size_t tc_smem_bytes(int D, int stages);   // bytes requested at launch (>= half an SM)
 int tc_rows();
 int tc_parts_per_block();
+int tc_unit_cost();                        // fixed cost of a unit, in tiles, for the shares
 cudaError_t tc_prepare(int D, int stages, int ctas);
 cudaError_t launch_split_tc(const Params &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                             const CUtensorMap &tm_v, int stages, int ctas, cudaStream_t stream);

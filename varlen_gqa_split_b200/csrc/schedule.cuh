@@ -38,10 +38,16 @@ struct SeqLen {
     int q0, Lq, k0, Lk, tpu;
 };
 
+// tpu is the unit's weight in the flattened space: its tiles plus
+// p.unit_cost tiles' worth for what a unit costs besides its tiles (the
+// query load, the pipeline drain, the epilogue), so that blocks whose shares
+// hold many small units get fewer tiles.  A unit's real tile t sits at
+// position unit_cost + t of its range.
 __device__ __forceinline__ SeqLen seq_len(const Params &p, int b, bool report) {
     SeqLen s;
     const bool ok = load_lengths(p, b, report, s.q0, s.Lq, s.k0, s.Lk);
     s.tpu = unit_tiles(s.Lq, s.Lk, ok);
+    if (s.tpu > 0) s.tpu += p.unit_cost;
     return s;
 }
 
@@ -49,7 +55,7 @@ __device__ __forceinline__ SeqLen seq_len(const Params &p, int b, bool report) {
 struct Segment {
     int b, hk;
     SeqLen s;
-    int t0, t1;           // tiles [t0, t1) of the unit's tpu tiles
+    int t0, t1;           // positions [t0, t1) of the unit's tpu (weighted) positions
     long long Pu;         // global index of the unit's first tile
 };
 
@@ -262,7 +268,8 @@ __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long lo
         if (!begin(seg, role)) return false;
         const int ntiles = (seg.s.Lk + kBN - 1) / kBN;
         if (role == 0 || !p.dynamic) {
-            const int tb = role == 0 ? 0 : seg.t0, te = role == 0 ? ntiles : min(ntiles, seg.t1);
+            const int tb = role == 0 ? 0 : max(0, seg.t0 - p.unit_cost);
+            const int te = role == 0 ? ntiles : min(ntiles, max(0, seg.t1 - p.unit_cost));
             for (int t = tb; t < te; ++t)
                 if (!tile(seg, t, t == te - 1)) return false;
             if (te <= tb && !none(seg)) return false;

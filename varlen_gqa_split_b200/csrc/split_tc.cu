@@ -670,6 +670,11 @@ size_t tc_smem_bytes(int D, int stages) {
 
 int tc_rows() { return kRows; }
 int tc_parts_per_block() { return kEpiWarps; }
+// A unit costs about three tiles' time besides its tiles (the query load, the
+// pipeline drain of its last tile and the epilogue), measured on the
+// short-query workload; the shares count it so that blocks holding many
+// small units take fewer tiles.
+int tc_unit_cost() { return 3; }
 
 cudaError_t tc_prepare(int D, int stages, int ctas) {
     void *fn = D == 64 ? tc_kernel_ptr<64>() : tc_kernel_ptr<128>();
