@@ -252,6 +252,37 @@ int attn_run_paged(attn_plan_t plan, const void *q, const void *k_cache, const v
                    const int32_t *cu_k, void *out, float *lse, void *stream);
 
 /*
+ * attn_merge_lse -- combine n attention results computed over disjoint key
+ * ranges of the same queries (context parallelism: each GPU attends over its
+ * own stretch of every sequence's keys; after an all-gather of the (out, lse)
+ * pairs every GPU merges them).  Asynchronous on `stream`, no sync, no
+ * allocation, capturable.
+ *
+ *   outs   device, bf16 [n_parts, T_q, Hq, D], 16-byte aligned: part r's out
+ *   lses   device, fp32 [n_parts, T_q, Hq], 4-byte aligned: part r's lse
+ *          (natural log, -inf where the part saw no key)
+ *   cu_q   device, int32, B_max + 1 entries: only tokens
+ *          [cu_q[0], cu_q[B_max]) are merged and written
+ *   out    device, bf16 [T_q, Hq, D]; lse device, fp32 [T_q, Hq]
+ *
+ * Per row: M = max_r lse_r, w_r = e^(lse_r - M), out = sum_r w_r out_r /
+ * sum_r w_r, lse = M + ln sum_r w_r; a row with every lse_r = -inf gets
+ * out = 0, lse = -inf.  The tail-aligned causal mask is a no-op at q_len = 1,
+ * so decode splits its keys anywhere; with q_len > 1 each part must have
+ * applied the mask for its keys' global positions (attn_run does so only for
+ * the part that holds the sequence's last keys).  Errors: NULL pointers,
+ * misalignment, sizes out of range (n_parts 1..65536, D 64 or 128); nothing
+ * is launched then.
+ *
+ * Source: the log-sum-exp merge of split partials (AstrAI commit log for
+ * csrc/kernels/gqa_decode_attn.cu, split-KV commit) and the reduction of the
+ * running (m, l, O) state between devices (kernbench2 docs/adr-proposed
+ * commit log, GQA entry), here as one all-gather and a local merge.
+ */
+int attn_merge_lse(int n_parts, const void *outs, const float *lses, int64_t T_q, const int32_t *cu_q,
+                   int B_max, int Hq, int D, void *out, float *lse, void *stream);
+
+/*
  * attn_check_error -- synchronise `stream`, then read and clear the plan's
  * sticky device error bits (ATTN_DEV_ERR_*) into *flags.  When a bit was set
  * it also resets the plan's merge tickets, so the plan stays usable after a

@@ -231,3 +231,24 @@ def attention_paged(q, k_cache, v_cache, block_table, page_size, cu_q, cu_k, *, 
     k, cu = gather_pages(k_cache, block_table, page_size, cu_k, B=B)
     v, _ = gather_pages(v_cache, block_table, page_size, cu_k, B=B)
     return attention(q, k, v, cu_q, cu, B=B, Hq=Hq, Hkv=Hkv, D=D, scale=scale, causal=causal)
+
+
+def merge_lse(outs, lses):
+    """Combine results over disjoint key ranges given as normalised pairs:
+    outs [n, ..., D] float64, lses [n, ...] (natural log, -inf for a part
+    with no key).  Per row M = max_r lse_r, w_r = exp(lse_r - M),
+    out = sum_r w_r out_r / sum_r w_r, lse = M + ln sum_r w_r; a row with no
+    key anywhere gives out = 0, lse = -inf (the log-sum-exp merge of split
+    partials, AstrAI commit log for csrc/kernels/gqa_decode_attn.cu, split-KV
+    commit, on normalised parts)."""
+    outs = np.asarray(outs, dtype=np.float64)
+    lses = np.asarray(lses, dtype=np.float64)
+    M = lses.max(axis=0)
+    finite = np.isfinite(M)
+    Mref = np.where(finite, M, 0.0)
+    w = np.where(np.isfinite(lses), np.exp(lses - Mref[None]), 0.0)
+    L = w.sum(axis=0)
+    out = np.where(finite[..., None], (w[..., None] * np.nan_to_num(outs)).sum(axis=0) /
+                   np.where(L > 0, L, 1.0)[..., None], 0.0)
+    lse = np.where(finite, Mref + np.log(np.where(L > 0, L, 1.0)), -np.inf)
+    return out, lse

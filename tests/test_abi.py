@@ -33,7 +33,7 @@ def libvgqa():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_run_strided", "attn_run_paged",
-              "attn_check_error", "attn_destroy", "attn_strerror", "attn_run_noalloc"):
+              "attn_merge_lse", "attn_check_error", "attn_destroy", "attn_strerror", "attn_run_noalloc"):
         assert n in names
 
 
@@ -78,6 +78,9 @@ def test_strerror_and_host_errors_without_gpu(libvgqa):
                                    [ctypes.c_void_p, ctypes.c_int] + [ctypes.c_void_p] * 5)
     assert lib.attn_run_paged(None, None, None, None, 2048, 256, 16, 4, None, 8, None, None, None, None,
                               None) == -5
+    lib.attn_merge_lse.argtypes = ([ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p] +
+                                   [ctypes.c_int] * 3 + [ctypes.c_void_p] * 3)
+    assert lib.attn_merge_lse(2, None, None, 4, None, 1, 8, 128, None, None, None) == -3   # no GPU touched
     lib.attn_plan_info.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     buf = ctypes.create_string_buffer(256)
     assert lib.attn_plan_info(ctypes.c_void_p(0x1234), buf) == -5          # unknown handle

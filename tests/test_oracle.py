@@ -557,3 +557,45 @@ def test_gather_pages_rejects_a_page_outside_the_cache():
     bt[1, 2] = pc.k_cache.shape[0]                  # sequence 1 has 70 keys: its third page is used
     with pytest.raises(ValueError):
         oracle.gather_pages(W.bits(pc.k_cache), bt, 16, batch.cu_k, B=sh.B)
+
+
+# ------------------------------------------------------------ merge of normalised parts
+
+@pytest.mark.parametrize("n_parts", [1, 2, 3, 7])
+def test_merge_lse_of_key_ranges_equals_whole(n_parts):
+    """Attention over disjoint key ranges of each sequence (some ranges empty,
+    one sequence without keys), merged from (out, lse) pairs, equals the
+    attention over all keys."""
+    sh = W.Shape("cp", B=5, Hq=8, Hkv=2, D=64, max_q=1, s_max=300)
+    lk = [300, 5, 0, 2, 77]
+    batch = W.make_batch(sh, [1] * 5, lk, seed=11)
+    q, k, v = W.bits(batch.q), W.bits(batch.k), W.bits(batch.v)
+    ref_o, ref_l = oracle.attention(q, k, v, batch.cu_q, batch.cu_k, B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D)
+    outs, lses = [], []
+    for r in range(n_parts):
+        sel, lens = [], []
+        for b in range(sh.B):
+            a = int(batch.cu_k[b]) + lk[b] * r // n_parts
+            e = int(batch.cu_k[b]) + lk[b] * (r + 1) // n_parts
+            sel.extend(range(a, e))
+            lens.append(e - a)
+        cu = W.cu_from_lengths(np.array(lens))
+        o, l = oracle.attention(q, k[sel], v[sel], batch.cu_q, cu, B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D)
+        outs.append(o)
+        lses.append(l)
+    o, l = oracle.merge_lse(np.stack(outs), np.stack(lses))
+    assert np.abs(o - ref_o).max() < 1e-12
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(np.isneginf(l), np.isneginf(ref_l))
+    assert np.abs(l[fin] - ref_l[fin]).max() < 1e-12
+    assert np.all(o[~fin] == 0.0)
+
+
+def test_merge_lse_weights_by_exponentiated_lse():
+    """Two parts with lse ln 1 and ln 3 (weights 1/4 and 3/4), and a part
+    with no key, which is ignored."""
+    outs = np.array([[[1.0, 0.0]], [[0.0, 4.0]], [[np.nan, np.nan]]])
+    lses = np.array([[0.0], [np.log(3.0)], [-np.inf]])
+    o, l = oracle.merge_lse(outs, lses)
+    assert np.allclose(o, [[0.25, 3.0]], atol=1e-15, rtol=0)
+    assert abs(l[0] - np.log(4.0)) < 1e-15

@@ -11,8 +11,9 @@ only marshals torch tensors into it.
 """
 from ._binding import (ATTN_COMBINE_AUTO, ATTN_COMBINE_FUSED, ATTN_COMBINE_KERNEL, ATTN_DEV_ERR_K_TOO_LONG, ATTN_DEV_ERR_OFFSETS, ATTN_DEV_ERR_PAGE, ATTN_DEV_ERR_Q_TOO_LONG,
                        ATTN_DEV_ERR_TIMEOUT, ATTN_VARIANT_AUTO, ATTN_VARIANT_MMA, ATTN_VARIANT_SIMT, ATTN_VARIANT_TC,
-                       AttnError, Plan, lib, strerror)
+                       AttnError, Plan, lib, merge_lse, strerror)
 
-__all__ = ["ATTN_COMBINE_AUTO", "ATTN_COMBINE_FUSED", "ATTN_COMBINE_KERNEL", "Plan", "AttnError", "lib", "strerror", "ATTN_VARIANT_AUTO", "ATTN_VARIANT_SIMT",
+__all__ = ["ATTN_COMBINE_AUTO", "ATTN_COMBINE_FUSED", "ATTN_COMBINE_KERNEL", "Plan", "AttnError", "lib", "merge_lse",
+           "strerror", "ATTN_VARIANT_AUTO", "ATTN_VARIANT_SIMT",
            "ATTN_VARIANT_MMA", "ATTN_VARIANT_TC", "ATTN_DEV_ERR_OFFSETS", "ATTN_DEV_ERR_Q_TOO_LONG",
            "ATTN_DEV_ERR_K_TOO_LONG", "ATTN_DEV_ERR_TIMEOUT", "ATTN_DEV_ERR_PAGE"]

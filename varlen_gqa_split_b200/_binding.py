@@ -27,7 +27,7 @@ ATTN_DEV_ERR_TIMEOUT = 0x8
 ATTN_DEV_ERR_PAGE = 0x10
 
 EXPORTED = ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_run_strided", "attn_run_paged",
-            "attn_check_error", "attn_destroy", "attn_strerror")
+            "attn_merge_lse", "attn_check_error", "attn_destroy", "attn_strerror")
 
 
 class Overrides(ctypes.Structure):
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         i64 = ctypes.c_int64
         L.attn_run_paged.argtypes = [vp, vp, vp, vp, i64, i64, i, i, i32p, i, i32p, i32p, vp, vp, vp]
         L.attn_run_paged.restype = i
+        L.attn_merge_lse.argtypes = [i, vp, vp, i64, i32p, i, i, i, vp, vp, vp]
+        L.attn_merge_lse.restype = i
         L.attn_check_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.attn_check_error.restype = i
         L.attn_destroy.argtypes = [vp]
@@ -86,6 +88,35 @@ def lib() -> ctypes.CDLL:
         L.attn_strerror.restype = ctypes.c_char_p
         _lib = L
         return L
+
+
+def merge_lse(outs, lses, cu_q, out=None, lse=None, stream=None):
+    """out, lse = merge_lse(outs, lses, cu_q[, out, lse, stream]): combine the
+    attention results of n disjoint key ranges (attn_merge_lse).
+
+    outs [n, T_q, Hq, D] bf16 and lses [n, T_q, Hq] fp32 contiguous CUDA
+    tensors; cu_q int32 [B_max + 1]; only tokens [cu_q[0], cu_q[B_max]) are
+    written."""
+    if outs.dtype != torch.bfloat16 or not outs.is_cuda or not outs.is_contiguous() or outs.dim() != 4:
+        raise ValueError("outs must be a contiguous bf16 CUDA tensor [n, T_q, Hq, D]")
+    n, T_q, Hq, D = outs.shape
+    if lses.dtype != torch.float32 or not lses.is_contiguous() or tuple(lses.shape) != (n, T_q, Hq):
+        raise ValueError("lses must be a contiguous fp32 tensor [n, T_q, Hq]")
+    if cu_q.dtype != torch.int32 or not cu_q.is_cuda or not cu_q.is_contiguous() or cu_q.dim() != 1:
+        raise ValueError("cu_q must be a contiguous int32 CUDA tensor")
+    if out is None:
+        out = torch.empty(T_q, Hq, D, dtype=torch.bfloat16, device=outs.device)
+    if lse is None:
+        lse = torch.empty(T_q, Hq, dtype=torch.float32, device=outs.device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (T_q, Hq, D) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor [T_q, Hq, D]")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (T_q, Hq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor [T_q, Hq]")
+    rc = lib().attn_merge_lse(int(n), outs.data_ptr(), lses.data_ptr(), int(T_q), cu_q.data_ptr(),
+                              int(cu_q.numel() - 1), int(Hq), int(D), out.data_ptr(), lse.data_ptr(),
+                              _stream_ptr(stream))
+    _check(rc, "attn_merge_lse")
+    return out, lse
 
 
 def strerror(code: int) -> str:
