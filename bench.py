@@ -53,7 +53,21 @@ DESCRIPTIONS = {
                   "sigma 1) in [1,16384], step 0",
     "shortq": "short-query varlen: B=32, q_len~U{1..16}, Hq=32, Hkv=4, D=128, kv~U{q_len..4096}, causal",
     "tiny": "tiny decode: B=2, q_len=1, Hq=4, Hkv=1, D=64, kv={37,100}",
+    "prefill": "causal prefill (queries longer than one 128-row tile): B=4, q_len=kv~U{512..2048}, Hq=32, "
+               "Hkv=4, D=128",
 }
+
+
+def attention_flops(batch: W.Batch) -> int:
+    """4 * D flops per visible (query, key) pair and query head (S = Q K^T and
+    P V), with the tail-aligned causal mask."""
+    sh = batch.shape
+    pairs = 0
+    for lq, lk in zip(batch.lens_q.tolist(), batch.lens_k.tolist()):
+        # query qi sees min(lk, max(0, lk - lq + qi + 1)) keys
+        for qi in range(int(lq)):
+            pairs += min(int(lk), max(0, int(lk) - int(lq) + qi + 1))
+    return 4 * sh.D * sh.Hq * pairs
 
 
 def algorithmic_bytes(batch: W.Batch) -> dict:
@@ -146,6 +160,16 @@ def measured_peak():
         return float(j["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
     except Exception:
         return 6650.0, "fallback 6.65 TB/s (pool measurement)"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor peak: the burst figure of a cuBLAS GEMM timed alone."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            j = json.load(f)
+        return float(j["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except Exception:
+        return 1590.0, "fallback 1.59 PFLOP/s (pool measurement)"
 
 
 def kernel_source_hash() -> str:
@@ -470,6 +494,15 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
                           if launches_per_call == 2 else "one call: the split kernel alone")}
     if traffic is None:
         roofline["traffic_note"] = traffic_note
+    if args.workload == "prefill":
+        # queries of up to 2048 tokens: the contraction, not HBM, bounds it
+        flops = attention_flops(batch)
+        tpeak, tsrc = measured_tensor_peak()
+        tach = flops / (total_ms / args.steps * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": kernel, "achieved": tach, "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": tach / tpeak, "traffic": traffic, "peak_source": tsrc,
+                    "algorithmic_flops_per_launch": flops, "hbm_gbs": achieved,
+                    "timed": roofline["timed"]}
 
     # end to end through the public API with pinned host buffers
     e2e = None

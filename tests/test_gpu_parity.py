@@ -421,7 +421,7 @@ def test_host_side_errors_launch_nothing():
     with pytest.raises(vg.AttnError):
         vg.Plan(1, 64, 64, 8, 128, 4, variant=MMA)         # 32 rows > warp-MMA path limit
     with pytest.raises(vg.AttnError):
-        vg.Plan(1, 64, 64, 8, 128, 17, variant=TC)         # 136 rows > tcgen05 path limit
+        vg.Plan(1, 64, 256, 1, 64, 1, variant=TC)          # G = 256 heads of one token exceed a 128-row tile
     with pytest.raises(vg.AttnError):
         vg.Plan(1, 64, 8, 1, 128, 1, variant=MMA, nsplit=2)  # split count belongs to the SIMT grid
     handle = plan.handle
@@ -430,3 +430,44 @@ def test_host_side_errors_launch_nothing():
                       out.data_ptr(), lse.data_ptr(), s) == -5
     torch.cuda.synchronize()
     assert torch.all(out == 0)
+
+
+# ------------------------------------------------------------ long queries (row tiles on tcgen05)
+
+@pytest.mark.parametrize("Hq,Hkv,D,max_q", [(16, 2, 128, 100), (40, 8, 128, 60), (8, 8, 64, 300),
+                                            (32, 2, 128, 33), (16, 1, 64, 40)])
+def test_tc_row_tiles_long_queries(Hq, Hkv, D, max_q):
+    """Queries longer than one 128-row tile: each sequence's queries are cut
+    into row tiles of 128 / G tokens from its end, each its own unit with the
+    keys its last token sees under the tail-aligned causal mask.  Includes
+    Lq > Lk (leading queries that see no key), Lq = 1, an empty sequence and
+    a partial first row tile."""
+    G = Hq // Hkv
+    lq = [max_q, min(37, max_q), 1, max_q // 2 + 1, 0, 7]
+    lk = [1000, 37, 5, 20, 9, 0]
+    sh = W.Shape("rowtiles", B=len(lq), Hq=Hq, Hkv=Hkv, D=D, max_q=max_q, s_max=1000)
+    batch = W.make_batch(sh, lq, lk, seed=29, gen_device="cuda")
+    ref_o, ref_l = oracle_full(batch)
+    cov = covered_rows(batch)
+    for kw in ({}, {"ctas": 5}, {"ctas": 5, "deterministic": 1}):
+        plan = plan_for(sh, **kw)
+        assert plan.info["variant"] == TC, plan.info
+        out, lse = run_gpu(plan, batch, extra_q_rows=2)
+        compare_full(out, lse, ref_o, ref_l, cov)
+
+
+@pytest.mark.parametrize("variant", [0, SIMT])
+def test_prefill_workload_sampled(variant):
+    """Causal prefill (q_len = kv_len up to 2048, G = 8: 128 row tiles of 16
+    tokens per sequence and KV head) against the oracle on sampled rows, and
+    the sentinel rows past cu_q untouched."""
+    batch = W.workload("prefill", gen_device="cuda")
+    sh = batch.shape
+    plan = plan_for(sh, variant=variant)
+    assert plan.info["variant"] == (variant or TC)
+    out, lse = run_gpu(plan, batch, extra_q_rows=3)
+    rng = np.random.default_rng(4)
+    rows = sample_rows(batch, 300, rng)
+    compare_rows(out, lse, batch, rows)
+    raw = out.view(torch.int16).numpy()
+    assert np.all(raw[int(batch.cu_q[-1]):] == np.int16(0x7FC0))

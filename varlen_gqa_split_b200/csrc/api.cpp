@@ -34,6 +34,8 @@ struct attn_plan_s {
     uint32_t *ticket;          // fused-merge arrival counters
     size_t ticket_bytes;
     int merge_bytes;           // tensor-core path: shared bytes of the merge area
+    int qtile;                 // tensor-core path: query tokens per row tile
+    int max_rt;                // tensor-core path: row tiles per sequence at most
     float *o_part;
     float2 *ml_part;
 };
@@ -96,14 +98,14 @@ int encode_paged_map(CUtensorMap *map, const void *base, int Hkv, int D, int pag
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
 }
 
-// [T, Hq, D] bf16, box = 64 elements x G heads x max_q tokens: one unit's
+// [T, Hq, D] bf16, box = 64 elements x G heads x qtile tokens: one unit's
 // query rows (token-major, heads inner) as the tcgen05 kernel's A operand.
 // Loads are right-aligned to the sequence's last query token, so, as for K/V,
 // the token extent is left open.
-int encode_q_map(CUtensorMap *map, const void *base, int Hq, int D, int G, int max_q) {
+int encode_q_map(CUtensorMap *map, const void *base, int Hq, int D, int G, int qtile) {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)0x7fffffff};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)max_q};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)qtile};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -176,15 +178,17 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     d.num_sms = sms;
 
     // warp-MMA kernel up to 16 query rows per KV head (the rows ride on the
-    // MMA's n8 side), tcgen05 kernel up to 128 (the rows are the M = 128
-    // side), CUDA cores beyond
+    // MMA's n8 side); tcgen05 kernel beyond, 128 rows (the M = 128 side) per
+    // unit and longer queries in row tiles of 128 / G tokens; CUDA cores when
+    // a single token's G heads exceed 128 rows
+    const int G_ = Hq / Hkv;
     int variant = o && o->variant ? o->variant
                                   : (rows <= 16 ? ATTN_VARIANT_MMA
-                                                : (rows <= tc_rows() ? ATTN_VARIANT_TC : ATTN_VARIANT_SIMT));
+                                                : (G_ <= tc_rows() ? ATTN_VARIANT_TC : ATTN_VARIANT_SIMT));
     if (variant != ATTN_VARIANT_MMA && variant != ATTN_VARIANT_SIMT && variant != ATTN_VARIANT_TC)
         return ATTN_E_INVALID_ARG;
     if (variant == ATTN_VARIANT_MMA && rows > 16) return ATTN_E_UNSUPPORTED;
-    if (variant == ATTN_VARIANT_TC && rows > tc_rows()) return ATTN_E_UNSUPPORTED;
+    if (variant == ATTN_VARIANT_TC && G_ > tc_rows()) return ATTN_E_UNSUPPORTED;
     if (o && o->block_n && o->block_n != 64) return ATTN_E_UNSUPPORTED;
     if (o && (o->nsplit < 0 || o->stages < 0 || o->ctas < 0)) return ATTN_E_INVALID_ARG;
     if (o && o->combine && o->combine != ATTN_COMBINE_KERNEL && o->combine != ATTN_COMBINE_FUSED)
@@ -193,6 +197,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     const int tiles_max = (s_max + 63) / 64;
 
     int NT = 1;
+    int qtile = max_q, max_rt = 1;
     size_t n_ticket = 0, n_part = 0, part_rows = 0;
     int merge_bytes = 0;
     if (variant == ATTN_VARIANT_MMA || variant == ATTN_VARIANT_TC) {
@@ -203,7 +208,11 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         const bool tcv = variant == ATTN_VARIANT_TC;
         NT = rows <= 8 ? 1 : 2;
         d.block_n = mma_block_n();
-        const long long max_tiles = (long long)B_max * Hkv * tiles_max;
+        if (tcv) {
+            qtile = std::min(max_q, tc_rows() / (Hq / Hkv));
+            max_rt = (max_q + qtile - 1) / qtile;
+        }
+        const long long max_tiles = (long long)B_max * Hkv * max_rt * tiles_max;
         long long ctas = o && o->ctas ? o->ctas : sms;
         ctas = std::min<long long>(ctas, std::max(1LL, max_tiles));
         ctas = std::min<long long>(ctas, 65535);
@@ -225,8 +234,8 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         d.grid_z = 1;
         d.deterministic = o && o->deterministic ? 1 : 0;
         d.combine = ATTN_COMBINE_KERNEL;     // slot-parallel combine, programmatic dependent launch
-        d.combine_blocks = 2 * d.ctas * combine_slots_split((int)rows, D);
-        n_ticket = 3 * (size_t)B_max * Hkv;  // per cut unit: tile claims (64-bit), part count
+        d.combine_blocks = 2 * d.ctas * combine_slots_split((Hq / Hkv) * qtile, D);
+        n_ticket = 3 * (size_t)B_max * Hkv * max_rt;   // per unit: tile claims (64-bit), part count
         n_part = 2 * (size_t)d.ctas;       // two partial slots per block
         part_rows = d.rows_per_block;
         if ((tcv ? tc_prepare(D, stages, d.ctas) : mma_prepare(D, NT, stages, d.ctas)) != cudaSuccess)
@@ -289,6 +298,8 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     p->device = dev;
     p->NT = NT;
     p->merge_bytes = merge_bytes;
+    p->qtile = qtile;
+    p->max_rt = max_rt;
     p->scale_log2 = (float)((1.0 / std::sqrt((double)D)) * 1.4426950408889634);
     if (cudaMalloc(&p->scratch, total) != cudaSuccess) {
         cudaGetLastError();
@@ -412,7 +423,7 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     }
     p.ticket = plan->ticket;
     p.claim = reinterpret_cast<unsigned long long *>(plan->ticket);
-    p.done = plan->ticket + 2 * (size_t)d.B_max * d.Hkv;
+    p.done = plan->ticket + 2 * (size_t)d.B_max * d.Hkv * plan->max_rt;
     p.fused = d.combine == ATTN_COMBINE_FUSED;
     p.merge_bytes = plan->merge_bytes;
     p.ctas_max = d.ctas;
@@ -421,6 +432,8 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     p.dynamic = persistent && !d.deterministic;
     p.done_per_part = d.variant == ATTN_VARIANT_TC ? tc_parts_per_block() : 1;
     p.unit_cost = d.variant == ATTN_VARIANT_TC ? tc_unit_cost() : 0;
+    p.qtile = plan->qtile;
+    p.max_rt = plan->max_rt;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(d.grid_x, d.grid_y, d.grid_z);
@@ -447,7 +460,7 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
         e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, d.ctas, s);
     } else if (d.variant == ATTN_VARIANT_TC) {
         CUtensorMap tm_q, tm_k, tm_v;
-        if (encode_q_map(&tm_q, q, d.Hq, d.D, d.G, d.max_q) != ATTN_OK || !kv_maps(tm_k, tm_v))
+        if (encode_q_map(&tm_q, q, d.Hq, d.D, d.G, plan->qtile) != ATTN_OK || !kv_maps(tm_k, tm_v))
             return ATTN_E_CUDA;
         e = launch_split_tc(p, tm_q, tm_k, tm_v, d.stages, d.ctas, s);
     } else {

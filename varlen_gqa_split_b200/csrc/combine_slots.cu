@@ -67,17 +67,21 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
         while (wk.next(p, seg)) ++nseg;
         if (nseg == 1) return;
     }
-    if (seg.t0 == 0 && seg.t1 == seg.s.tpu) return;   // whole unit: written by the split kernel
+    if (seg.t0 == 0 && seg.t1 == seg.w) return;       // whole unit: written by the split kernel
     const long long T = sh.T;
     const int Ce = sh.Ce;
     const int c_first = block_of(seg.Pu, T, Ce);
-    const int n = block_of(seg.Pu + seg.s.tpu - 1, T, Ce) - c_first + 1;
-    const int G = p.G, R = G * seg.s.Lq;
+    const int n = block_of(seg.Pu + seg.w - 1, T, Ce) - c_first + 1;
+    // the row tile's tokens [tq0, tq0 + nq) of the sequence; partial row r is
+    // token tq0 + r / G, head r % G of the KV head's group
+    const int tq0 = rt_first(seg.s, seg.rt, p.qtile);
+    const int nq = seg.s.Lq - seg.rt * p.qtile - tq0;
+    const int G = p.G, R = G * nq;
     const int items = R * kCols;
     const int nb = n * S;                          // blocks merging this unit
     const int per = (items + nb - 1) / nb;
     const int it_lo = min(items, ((c - c_first) * S + sub) * per), it_hi = min(items, it_lo + per);
-    const long long u = (long long)seg.b * p.Hkv + seg.hk;
+    const long long u = unit_index(p, seg.b, seg.hk, seg.rt);
 
     int *slots = reinterpret_cast<int *>(csm);                         // [n]
     for (int j = tid; j < n; j += kT) slots[j] = slot_of(c_first + j, seg.Pu, T, Ce);
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
 
     auto write_row = [&](int r, int d4, float Mt, float Lt, float4 acc) {
         const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
-        const int qi = r / G, h = seg.hk * G + r % G;
+        const int qi = tq0 + r / G, h = seg.hk * G + r % G;
         const long long tok = seg.s.q0 + qi;
         uint2 pk;
         pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);

@@ -35,6 +35,8 @@ struct Params {
     int done_per_part;         // tensor-core path: releases on `done` per written part
     int share_stride;          // tensor-core path: block b takes share (b * share_stride) mod blocks
     int unit_cost;             // tensor-core path: tiles' worth of fixed cost per unit in the shares
+    int qtile;                 // tensor-core path: query tokens per row tile (a unit is (b, hk, row tile))
+    int max_rt;                // tensor-core path: row tiles of a sequence at most (counter stride)
     long long k_stride;        // elements between consecutive tokens of k (Hkv * D when packed)
     long long v_stride;        // elements between consecutive tokens of v
     // paged K/V (block_table != null): key j of sequence b sits in page

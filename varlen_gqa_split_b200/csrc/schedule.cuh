@@ -2,8 +2,12 @@
 // split kernels and the slot combine kernel (device code, internal).
 //
 // The work is the flattened sequence of 64-key tiles of every unit
-// u = (sequence b, KV head hk), in order of b then hk; a unit with queries but
-// no keys counts as one (empty) tile so that it still gets its defined output.
+// u = (sequence b, KV head hk, row tile rt), in order of b, hk, rt.  A row tile
+// holds p.qtile query tokens (all of a decode sequence's; for long queries
+// the tokens are tiled from the sequence's end, so tile rt ends qtile * rt
+// tokens before it) and needs the keys its last token sees under the
+// tail-aligned causal mask.  A unit whose rows see no key counts as one
+// (empty) tile so that it still gets its defined output.
 // Each of the C blocks (C fixed by the plan, about one per SM) takes the
 // contiguous, equal share [c*T/C, (c+1)*T/C) of the T tiles, computed on the
 // device from cu_seqlens at the start of every call -- no host round trip and
@@ -27,77 +31,126 @@ namespace sched {
 constexpr int kBN = 64;                   // keys per tile
 constexpr int kClaim = 2;                 // tiles per claim on a shared unit's counter
 
-// tiles of one unit of sequence b: 0 if the sequence is skipped (no query
-// rows, or lengths outside the plan), else max(1, ceil(Lk / 64))
-__device__ __forceinline__ int unit_tiles(int Lq, int Lk, bool ok) {
-    if (!ok || Lq <= 0) return 0;
-    return Lk > 0 ? (Lk + kBN - 1) / kBN : 1;
-}
-
 struct SeqLen {
-    int q0, Lq, k0, Lk, tpu;
+    int q0, Lq, k0, Lk;
+    int nrt;              // row tiles (0: the sequence is skipped)
+    int tpu;              // weighted positions of one KV head: sum over its row tiles of unit_weight
 };
 
-// tpu is the unit's weight in the flattened space: its tiles plus
-// p.unit_cost tiles' worth for what a unit costs besides its tiles (the
-// query load, the pipeline drain, the epilogue), so that blocks whose shares
-// hold many small units get fewer tiles.  A unit's real tile t sits at
-// position unit_cost + t of its range.
+// key tiles of row tile rt: ceil(keys its last token sees / 64), 0 if none
+__device__ __forceinline__ int rt_tiles(const SeqLen &s, int rt, int qtile) {
+    const int vis = s.Lk - rt * qtile;
+    return vis > 0 ? (vis + kBN - 1) / kBN : 0;
+}
+
+// A unit's weight in the flattened space: its tiles (at least one, the
+// empty tile of a unit that sees no key) plus p.unit_cost tiles' worth for
+// what a unit costs besides its tiles (the query load, the pipeline drain,
+// the epilogue), so that blocks whose shares hold many small units get fewer
+// tiles.  A unit's real tile t sits at position unit_cost + t of its range.
+__device__ __forceinline__ int unit_weight(const Params &p, int tiles) { return max(tiles, 1) + p.unit_cost; }
+
 __device__ __forceinline__ SeqLen seq_len(const Params &p, int b, bool report) {
     SeqLen s;
     const bool ok = load_lengths(p, b, report, s.q0, s.Lq, s.k0, s.Lk);
-    s.tpu = unit_tiles(s.Lq, s.Lk, ok);
-    if (s.tpu > 0) s.tpu += p.unit_cost;
+    if (!ok || s.Lq <= 0) {
+        s.nrt = s.tpu = 0;
+    } else if (s.Lq <= p.qtile) {                 // one row tile: every decode sequence
+        s.nrt = 1;
+        s.tpu = unit_weight(p, rt_tiles(s, 0, p.qtile));
+    } else {
+        s.nrt = (s.Lq + p.qtile - 1) / p.qtile;
+        s.tpu = 0;
+        for (int rt = 0; rt < s.nrt; ++rt) s.tpu += unit_weight(p, rt_tiles(s, rt, p.qtile));
+    }
     return s;
 }
 
 // One stretch of a unit inside a block's share.
 struct Segment {
-    int b, hk;
+    int b, hk, rt;
     SeqLen s;
-    int t0, t1;           // positions [t0, t1) of the unit's tpu (weighted) positions
-    long long Pu;         // global index of the unit's first tile
+    int nt;               // the unit's key tiles
+    int w;                // its weight (positions)
+    int t0, t1;           // positions [t0, t1) of the unit's w positions
+    long long Pu;         // global index of the unit's first position
 };
+
+// counters of unit (b, hk, rt): tile claims, part counts
+__device__ __forceinline__ long long unit_index(const Params &p, int b, int hk, int rt) {
+    return ((long long)b * p.Hkv + hk) * p.max_rt + rt;
+}
+
+// token range [lo, lo + n) of row tile rt, and where its box starts (may be
+// before the sequence: those rows do not exist)
+__device__ __forceinline__ int rt_box_start(const SeqLen &s, int rt, int qtile) { return s.Lq - (rt + 1) * qtile; }
+__device__ __forceinline__ int rt_first(const SeqLen &s, int rt, int qtile) {
+    return max(0, rt_box_start(s, rt, qtile));
+}
 
 // Walks a block's share [g, hi) of the flattened tile space unit by unit.
 struct SegWalker {
-    int b, hk;
+    int b, hk, rt;
     SeqLen s;
-    long long pb;         // global index of tile 0 of (b, hk = 0)
+    int nt, w;            // the current unit's tiles and weight
+    long long Pu;         // global index of the current unit's first position
     long long g, hi;
+
+    __device__ void set_unit(const Params &p) {
+        nt = rt_tiles(s, rt, p.qtile);
+        w = unit_weight(p, nt);
+    }
 
     __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi_) {
         b = b_first;
-        pb = pb_first;
         s = seq_len(p, b, false);
-        hk = (int)((lo - pb) / s.tpu);
+        hk = (int)((lo - pb_first) / s.tpu);
+        Pu = pb_first + (long long)hk * s.tpu;
+        rt = 0;
+        set_unit(p);
+        if (s.nrt > 1) {
+            while (Pu + w <= lo) {        // the row tile holding lo
+                Pu += w;
+                ++rt;
+                set_unit(p);
+            }
+        }
         g = lo;
         hi = hi_;
     }
 
     __device__ bool next(const Params &p, Segment &seg) {
         if (g >= hi) return false;
-        const long long Pu = pb + (long long)hk * s.tpu;
         seg.b = b;
         seg.hk = hk;
+        seg.rt = rt;
         seg.s = s;
+        seg.nt = nt;
+        seg.w = w;
         seg.Pu = Pu;
         seg.t0 = (int)(g - Pu);
-        const long long end = min(hi, Pu + s.tpu);
+        const long long end = min(hi, Pu + w);
         seg.t1 = (int)(end - Pu);
         g = end;
-        if (g < hi && ++hk == p.Hkv) {
-            // next sequence with work; the share ends before the tiles do, so
-            // one exists (the bound only guards against reading past cu)
-            pb += (long long)p.Hkv * s.tpu;
-            hk = 0;
-            do {
-                if (++b >= p.B_max) {
-                    g = hi;
-                    break;
+        if (g < hi) {
+            Pu += w;
+            if (++rt == s.nrt) {
+                rt = 0;
+                if (++hk == p.Hkv) {
+                    // next sequence with work; the share ends before the
+                    // tiles do, so one exists (the bound only guards against
+                    // reading past cu)
+                    hk = 0;
+                    do {
+                        if (++b >= p.B_max) {
+                            g = hi;
+                            break;
+                        }
+                        s = seq_len(p, b, false);
+                    } while (s.tpu == 0);
                 }
-                s = seq_len(p, b, false);
-            } while (s.tpu == 0);
+            }
+            if (g < hi) set_unit(p);
         }
         return true;
     }
@@ -129,7 +182,7 @@ struct OrderedWalker {
             while (true) {
                 const long long g0 = wk.g;
                 if (!wk.next(p, s)) break;
-                const bool whole = s.t0 == 0 && s.t1 == s.s.tpu;
+                const bool whole = s.t0 == 0 && s.t1 == s.w;
                 if (whole) {
                     seg = s;
                     role = 0;
@@ -266,7 +319,7 @@ __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long lo
     int role;
     while (wk.next(p, seg, role)) {
         if (!begin(seg, role)) return false;
-        const int ntiles = (seg.s.Lk + kBN - 1) / kBN;
+        const int ntiles = seg.nt;
         if (role == 0 || !p.dynamic) {
             const int tb = role == 0 ? 0 : max(0, seg.t0 - p.unit_cost);
             const int te = role == 0 ? ntiles : min(ntiles, max(0, seg.t1 - p.unit_cost));
@@ -275,7 +328,7 @@ __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long lo
             if (te <= tb && !none(seg)) return false;
             continue;
         }
-        unsigned long long *claim = p.claim + (long long)seg.b * p.Hkv + seg.hk;
+        unsigned long long *claim = p.claim + unit_index(p, seg.b, seg.hk, seg.rt);
         const bool up = seg.t0 == 0;                       // static part at the unit's front
         const unsigned long long inc = up ? ((unsigned long long)kClaim << 32) : (unsigned long long)kClaim;
         auto range = [&](unsigned long long old, int &t_lo, int &t_hi) {

@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
         }
         named_sync(kBarConsumers, kConsumers);     // warp-merge buffers free for the next unit
         // publish the part: the combine block merging this unit waits for all n
-        if (!whole && tid == 0) red_add_release_gpu(p.done + (long long)cur.b * p.Hkv + cur.hk, 1u);
+        if (!whole && tid == 0) red_add_release_gpu(p.done + unit_index(p, cur.b, cur.hk, cur.rt), 1u);
 
         if (!has_nxt) break;
         cur = nxt;

@@ -1,6 +1,7 @@
 // split_tc.cu -- persistent TMA-fed split-KV kernel on the fifth-generation
 // tensor cores (tcgen05, accumulators in tensor memory) for short-query row
-// counts: up to 128 query rows (G * max_q) per KV head.
+// counts: 128 query rows (G heads x 128 / G query tokens) per unit, and
+// longer queries as several row tiles of the sequence, each its own unit.
 //
 // Same schedule as the warp-MMA kernel (schedule.cuh: equal shares of the
 // flattened 64-key tiles, cut units merged by the slot combine kernel), but
@@ -13,7 +14,7 @@
 //
 // Warp roles (320 threads):
 //   warp 9, one lane -- producer: loads each unit's Q tile (one TMA box of G
-//     heads x max_q tokens, right-aligned so it ends at the sequence's last
+//     heads x qtile tokens, right-aligned so it ends at the row tile's last
 //     query token; rows past the sequence's own tokens are never written)
 //     into one of two Q buffers, then streams the unit's K and V tiles into a
 //     ring of shared-memory stages exactly like the warp-MMA kernel;
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const int G = p.G, QT = p.max_q;
+    const int G = p.G, QT = p.qtile;                         // query tokens per row tile
 
     if (has_work && warp == kProducerWarp && lane == 0) {
         // ---------------------------------------------------------- producer
@@ -193,7 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const int qb = k & 1;
             if (k >= 2 && !wait_bar(&q_free[qb], ((k - 2) >> 1) & 1, stop, p)) return false;
             mbar_arrive_expect_tx(&q_full[qb], q_bytes);
-            const int t_end = sg.s.q0 + sg.s.Lq;             // box ends at the sequence's last query token
+            // the box ends at the row tile's last query token
+            const int t_end = sg.s.q0 + sg.s.Lq - sg.rt * QT;
 #pragma unroll
             for (int hf = 0; hf < L::kHalves; ++hf)
                 tma_load_3d(qbuf + qb * L::kQTile + hf * L::kQRegion, &tm_q, &q_full[qb], hf * 64, sg.hk * G,
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         while (ok && wk.next(p, seg, role)) {
             const int Lq = seg.s.Lq, Lk = seg.s.Lk;
             const int tq = r / G, g = r - tq * G;
-            const int qi = tq - (QT - Lq);                       // this row's query token in the sequence
+            const int qi = tq + rt_box_start(seg.s, seg.rt, QT); // this row's query token in the sequence
             const bool valid = tq < QT && qi >= 0;
             const int vis = valid ? Lk - Lq + qi + 1 : 0;        // keys [0, vis) visible (tail-aligned causal)
             // a warp none of whose 32 rows is a query row of this unit only
@@ -576,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             }
             const bool whole = role == 0;
             const int slot = role == 1 ? 2 * c : 2 * c + 1;
-            const int pr = qi * G + g;                            // row within the unit's G * Lq rows
+            const int pr = (qi - rt_first(seg.s, seg.rt, QT)) * G + g;   // row within the unit's partial
             const long long tok = seg.s.q0 + qi;
             const int h = seg.hk * G + g;
             const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
@@ -629,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             // kEpiWarps writer warps of each of the unit's n blocks)
             if (!whole) {
                 __syncwarp();
-                if (lane == 0) red_add_release_gpu(p.done + (long long)seg.b * p.Hkv + seg.hk, 1u);
+                if (lane == 0) red_add_release_gpu(p.done + unit_index(p, seg.b, seg.hk, seg.rt), 1u);
             }
         }
         if (!ok) *stop = 1;

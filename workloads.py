@@ -15,6 +15,9 @@ design notes):
               kv ~ round(lognormal(mean 2048, sigma 1)) clamped to [1, 16384]
   shortq      B=32, q_len ~ U{1..16}, Hq=32, Hkv=4, D=128, kv ~ U{q_len..4096},
               tail-aligned causal mask
+  prefill     B=4, q_len = kv ~ U{512..2048}, Hq=32, Hkv=4, D=128, causal (queries
+              longer than one 128-row tile; not one of the method's five
+              workloads)
 
 Random streams: lengths come from ``numpy.random.default_rng(seed)`` (PCG64),
 one stream per workload, drawn in step order.  Values come from a
@@ -58,6 +61,9 @@ SHAPES = {
     "ragged": Shape("ragged", B=64, Hq=32, Hkv=8, D=128, max_q=1, s_max=8192),
     "continuous": Shape("continuous", B=256, Hq=64, Hkv=8, D=128, max_q=1, s_max=16384),
     "shortq": Shape("shortq", B=32, Hq=32, Hkv=4, D=128, max_q=16, s_max=4096),
+    # longer queries than one 128-row tile (G = 8: 16 tokens per row tile):
+    # causal prefill of whole sequences, q_len = kv_len ~ U{512..2048}
+    "prefill": Shape("prefill", B=4, Hq=32, Hkv=4, D=128, max_q=2048, s_max=2048),
 }
 
 CONTINUOUS_STEPS = 100
@@ -92,6 +98,9 @@ def lengths(name: str, seed: int = 0, steps: int | None = None):
         lq = rng.integers(1, 16, size=sh.B, endpoint=True)
         lk = np.array([rng.integers(int(a), 4096, endpoint=True) for a in lq], np.int64)
         return [(lq.astype(np.int64), lk)]
+    if name == "prefill":
+        lq = rng.integers(512, 2048, size=sh.B, endpoint=True).astype(np.int64)
+        return [(lq, lq.copy())]
     raise KeyError(name)
 
 
