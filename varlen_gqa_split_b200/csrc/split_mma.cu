@@ -61,7 +61,9 @@ __device__ __forceinline__ uint32_t swz(int row, int c) {
     return row * 128 + ((c ^ (row & 7)) << 4);
 }
 
-template <int D, int NT>
+// PAGED: K and V come from a paged cache (block table); a separate
+// instantiation keeps the packed kernel free of that code
+template <int D, int NT, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                 const __grid_constant__ CUtensorMap tm_v,
                                                                 const Params p, const int stages) {
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             };
             auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
                 const int ks = tile * kBN;
-                if (p.block_table && p.page_box == kBN && p.page_rows) {
+                if constexpr (PAGED) if (p.page_box == kBN && p.page_rows) {
                     // paged, pages of 64 keys or more a whole number of rows apart: one
                     // row index per tile, page * page_rows + slot, as lean as a packed
                     // tile (the table read is issued before the stage wait)
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                     advance();
                     return true;
                 }
-                if (p.block_table) {
+                if constexpr (PAGED) {
                     // paged, in general: the tile's keys in boxes of page_box keys,
                     // each from its page; the table is read before the stage wait,
                     // so the read overlaps it
@@ -230,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 return true;
             };
             auto begin = [&](const Segment &sg, int) -> bool {
-                if (p.block_table) prefetch_pages(p, sg.b, sg.s.Lk);
+                if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk);
                 return true;
             };
             feed_tiles(p, b_first, pb_first, lo, hi, begin, load_tile, empty_stage);
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             // key index of tile row 0: a packed tile past the sequence's end
             // was moved back to end at its last key; a paged tile starts at
             // t0, and its rows past Lk hold whatever the page held
-            const bool paged = p.block_table != nullptr;
+            constexpr bool paged = PAGED;
             const int ls = paged ? t0 : min(t0, Lk - kBN);
             bool zeroed = false;
             if (paged && t0 + kBN > Lk) {
@@ -504,13 +506,14 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
 }
 
 template <int D, int NT>
-void *mma_kernel_ptr() {
-    return reinterpret_cast<void *>(split_mma_kernel<D, NT>);
+void *mma_kernel_ptr(bool paged) {
+    return paged ? reinterpret_cast<void *>(split_mma_kernel<D, NT, true>)
+                 : reinterpret_cast<void *>(split_mma_kernel<D, NT, false>);
 }
 
-void *pick(int D, int NT) {
-    if (D == 64) return NT == 1 ? mma_kernel_ptr<64, 1>() : mma_kernel_ptr<64, 2>();
-    return NT == 1 ? mma_kernel_ptr<128, 1>() : mma_kernel_ptr<128, 2>();
+void *pick(int D, int NT, bool paged) {
+    if (D == 64) return NT == 1 ? mma_kernel_ptr<64, 1>(paged) : mma_kernel_ptr<64, 2>(paged);
+    return NT == 1 ? mma_kernel_ptr<128, 1>(paged) : mma_kernel_ptr<128, 2>(paged);
 }
 
 }  // namespace
@@ -536,8 +539,12 @@ int mma_block_n() { return kBN; }
 int mma_threads() { return kThreads; }
 
 cudaError_t mma_prepare(int D, int NT, int stages, int ctas) {
-    cudaError_t e = cudaFuncSetAttribute(pick(D, NT), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)mma_smem_bytes(D, NT, stages, ctas));
+    for (bool paged : {false, true}) {
+        const cudaError_t e = cudaFuncSetAttribute(pick(D, NT, paged), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)mma_smem_bytes(D, NT, stages, ctas));
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = cudaSuccess;
     if (e != cudaSuccess) return e;
     return combine_slots_prepare(D, ctas);
 }
@@ -562,7 +569,7 @@ cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUt
     int st = stages;
     void *split_args[] = {const_cast<CUtensorMap *>(&tm_k), const_cast<CUtensorMap *>(&tm_v),
                           const_cast<Params *>(&p), &st};
-    cudaError_t e = cudaLaunchKernelExC(&cfg, pick(p.D, NT), split_args);
+    cudaError_t e = cudaLaunchKernelExC(&cfg, pick(p.D, NT, p.block_table != nullptr), split_args);
     if (e != cudaSuccess) return e;
     return launch_combine_slots(p, ctas, stream);
 }

@@ -97,7 +97,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     return true;
 }
 
-template <int D>
+// PAGED: K and V come from a paged cache (block table); a separate
+// instantiation keeps the packed kernel free of that code
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                const __grid_constant__ CUtensorMap tm_k,
                                                                const __grid_constant__ CUtensorMap tm_v,
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             }
         };
         auto begin = [&](const Segment &sg, int) -> bool {
-            if (p.block_table) prefetch_pages(p, sg.b, sg.s.Lk);
+            if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk);
             const int qb = k & 1;
             if (k >= 2 && !wait_bar(&q_free[qb], ((k - 2) >> 1) & 1, stop, p)) return false;
             mbar_arrive_expect_tx(&q_full[qb], q_bytes);
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         };
         auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
             const int ks = tile * kBN;
-            if (p.block_table && p.page_box == kBN && p.page_rows) {
+            if constexpr (PAGED) if (p.page_box == kBN && p.page_rows) {
                 // paged, pages of 64 keys or more a whole number of rows apart: one
                 // row index per tile, page * page_rows + slot, as lean as a packed
                 // tile (the table read is issued before the stage wait)
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 advance();
                 return true;
             }
-            if (p.block_table) {
+            if constexpr (PAGED) {
                 // paged, in general: the tile's keys in boxes of page_box keys,
                 // each from its page; the table is read before the stage wait,
                 // so the read overlaps it
@@ -449,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 }
                 if (mt.y & kMetaEmpty) break;
                 has_tiles = true;
-                if (p.block_table && mt.x + kBN > Lk) {
+                if (PAGED && mt.x + kBN > Lk) {
                     // paged tile past the sequence's end: zero its V rows
                     // past Lk (weight 0 times a stale non-finite value would
                     // not be 0) before this warp's P is signalled; the stage
@@ -487,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 // mask and max of this half.  The scale (> 0) enters in the
                 // exp2 argument, so the raw maximum gives the scaled one; a
                 // masked score becomes -inf, whose weight is exactly 0.
-                const int ks = mt.x, ls = p.block_table ? ks : min(ks, Lk - kBN);   // key of column 0
+                const int ks = mt.x, ls = PAGED ? ks : min(ks, Lk - kBN);   // key of column 0
                 const int c0 = half * kHalfKeys;
                 const int lo_c = ks - ls - c0, hi_c = min(kHalfKeys, vis - ls - c0);   // visible [lo_c, hi_c)
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -647,8 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
 }
 
 template <int D>
-void *tc_kernel_ptr() {
-    return reinterpret_cast<void *>(split_tc_kernel<D>);
+void *tc_kernel_ptr(bool paged) {
+    return paged ? reinterpret_cast<void *>(split_tc_kernel<D, true>)
+                 : reinterpret_cast<void *>(split_tc_kernel<D, false>);
 }
 
 }  // namespace
@@ -679,9 +682,12 @@ int tc_parts_per_block() { return kEpiWarps; }
 int tc_unit_cost() { return 3; }
 
 cudaError_t tc_prepare(int D, int stages, int ctas) {
-    void *fn = D == 64 ? tc_kernel_ptr<64>() : tc_kernel_ptr<128>();
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(D, stages));
-    if (e != cudaSuccess) return e;
+    for (bool paged : {false, true}) {
+        void *fn = D == 64 ? tc_kernel_ptr<64>(paged) : tc_kernel_ptr<128>(paged);
+        const cudaError_t e =
+            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(D, stages));
+        if (e != cudaSuccess) return e;
+    }
     return combine_slots_prepare(D, ctas);
 }
 
@@ -701,7 +707,8 @@ cudaError_t launch_split_tc(const Params &p, const CUtensorMap &tm_q, const CUte
     int st = stages;
     void *args[] = {const_cast<CUtensorMap *>(&tm_q), const_cast<CUtensorMap *>(&tm_k),
                     const_cast<CUtensorMap *>(&tm_v), const_cast<Params *>(&p), &st};
-    cudaError_t e = cudaLaunchKernelExC(&cfg, p.D == 64 ? tc_kernel_ptr<64>() : tc_kernel_ptr<128>(), args);
+    const bool paged = p.block_table != nullptr;
+    cudaError_t e = cudaLaunchKernelExC(&cfg, p.D == 64 ? tc_kernel_ptr<64>(paged) : tc_kernel_ptr<128>(paged), args);
     if (e != cudaSuccess) return e;
     return launch_combine_slots(p, ctas, stream);
 }
