@@ -98,6 +98,39 @@ int encode_paged_map(CUtensorMap *map, const void *base, int Hkv, int D, int pag
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
 }
 
+// The warp-MMA kernel's K/V maps: the same tensors with the D / 64 halves of
+// a row as the outermost dimension (stride 128 bytes), so that one box of
+// 64 elements x 1 head x box_rows tokens x D / 64 halves fills a tile's
+// halves one after the other ([half][row][128 B], 128-byte swizzle) and a
+// tile row range takes one load instead of one per half.  Packed or paged
+// with pages a whole number of rows apart: {64, Hkv, rows, halves}; other
+// paged caches: {64, Hkv, page_size, num_pages, halves}.
+int encode_kv_map_halves(CUtensorMap *map, const void *base, int Hkv, int D, int box_rows, long long token_stride,
+                         long long rows) {
+    const int halves = D / 64;
+    cuuint64_t dims[4] = {64, (cuuint64_t)Hkv, (cuuint64_t)rows, (cuuint64_t)halves};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)token_stride * 2, 128};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, (cuuint32_t)halves};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
+}
+
+int encode_paged_map_halves(CUtensorMap *map, const void *base, int Hkv, int D, int page_size, int num_pages,
+                            long long token_stride, long long page_stride) {
+    const int halves = D / 64;
+    cuuint64_t dims[5] = {64, (cuuint64_t)Hkv, (cuuint64_t)page_size, (cuuint64_t)num_pages, (cuuint64_t)halves};
+    cuuint64_t strides[4] = {(cuuint64_t)D * 2, (cuuint64_t)token_stride * 2, (cuuint64_t)page_stride * 2, 128};
+    cuuint32_t box[5] = {64, 1, (cuuint32_t)std::min(page_size, 64), 1, (cuuint32_t)halves};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_E_CUDA;
+}
+
 // [T, Hq, D] bf16, box = 64 elements x G heads x qtile tokens: one unit's
 // query rows (token-major, heads inner) as the tcgen05 kernel's A operand.
 // Loads are right-aligned to the sequence's last query token, so, as for K/V,
@@ -456,7 +489,19 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     cudaError_t e;
     if (d.variant == ATTN_VARIANT_MMA) {
         CUtensorMap tm_k, tm_v;
-        if (!kv_maps(tm_k, tm_v)) return ATTN_E_CUDA;
+        bool ok;
+        if (pg && !p.page_rows)
+            ok = encode_paged_map_halves(&tm_k, k, d.Hkv, d.D, pg->page_size, pg->num_pages, k_stride,
+                                         pg->page_stride) == ATTN_OK &&
+                 encode_paged_map_halves(&tm_v, v, d.Hkv, d.D, pg->page_size, pg->num_pages, v_stride,
+                                         pg->page_stride) == ATTN_OK;
+        else {
+            const long long rows = pg ? (long long)pg->num_pages * p.page_rows : 0x7fffffffll;
+            const int box = pg ? std::min(pg->page_size, 64) : d.block_n;
+            ok = encode_kv_map_halves(&tm_k, k, d.Hkv, d.D, box, k_stride, rows) == ATTN_OK &&
+                 encode_kv_map_halves(&tm_v, v, d.Hkv, d.D, box, v_stride, rows) == ATTN_OK;
+        }
+        if (!ok) return ATTN_E_CUDA;
         e = launch_split_mma(p, tm_k, tm_v, plan->NT, d.stages, d.ctas, s);
     } else if (d.variant == ATTN_VARIANT_TC) {
         CUtensorMap tm_q, tm_k, tm_v;

@@ -56,11 +56,6 @@ struct MmaLayout {
     static constexpr int kStageBytes = 2 * kTileBytes;      // K + V
 };
 
-// byte offset of (row, 16-byte chunk c) inside a 128B-swizzled [rows][128 B] region
-__device__ __forceinline__ uint32_t swz(int row, int c) {
-    return row * 128 + ((c ^ (row & 7)) << 4);
-}
-
 // PAGED: K and V come from a paged cache (block table); a separate
 // instantiation keeps the packed kernel free of that code
 template <int D, int NT, bool PAGED>
@@ -157,12 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                     meta[s] = make_int2(ks, last ? kMetaLast : 0);
                     uint8_t *st = ring + s * L::kStageBytes;
                     mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-#pragma unroll
-                    for (int hf = 0; hf < L::kHalves; ++hf)
-                        tma_load_3d(st + hf * L::kRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
-#pragma unroll
-                    for (int hf = 0; hf < L::kHalves; ++hf)
-                        tma_load_3d(st + L::kTileBytes + hf * L::kRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
+                    tma_load_4d(st, &tm_k, &full[s], 0, sg.hk, row, 0, pol);          // all halves
+                    tma_load_4d(st + L::kTileBytes, &tm_v, &full[s], 0, sg.hk, row, 0, pol);
                     advance();
                     return true;
                 }
@@ -195,16 +186,15 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                         // outside the map: zeros
                         const int page = (live >> i) & 1u ? page_checked(p, pg[i]) : p.num_pages;
                         const int slot = (ks + i * p.page_box) & slot_mask;   // 0 when pages are < 64 keys
-#pragma unroll
-                        for (int hf = 0; hf < L::kHalves; ++hf) {
-                            uint8_t *dk = st + hf * L::kRegion + i * p.page_box * 128, *dv = dk + L::kTileBytes;
-                            if (p.page_rows) {
-                                tma_load_3d(dk, &tm_k, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
-                                tma_load_3d(dv, &tm_v, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
-                            } else {
-                                tma_load_4d(dk, &tm_k, &full[s], hf * 64, sg.hk, slot, page, pol);
-                                tma_load_4d(dv, &tm_v, &full[s], hf * 64, sg.hk, slot, page, pol);
-                            }
+                        // box i holds its page_box rows of every half:
+                        // [half][row][128 B] at i * page_box * D * 2
+                        uint8_t *dk = st + i * p.page_box * L::kHalves * 128, *dv = dk + L::kTileBytes;
+                        if (p.page_rows) {
+                            tma_load_4d(dk, &tm_k, &full[s], 0, sg.hk, page * p.page_rows + slot, 0, pol);
+                            tma_load_4d(dv, &tm_v, &full[s], 0, sg.hk, page * p.page_rows + slot, 0, pol);
+                        } else {
+                            tma_load_5d(dk, &tm_k, &full[s], 0, sg.hk, slot, page, 0, pol);
+                            tma_load_5d(dv, &tm_v, &full[s], 0, sg.hk, slot, page, 0, pol);
                         }
                     }
                     advance();
@@ -215,12 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 meta[s] = make_int2(ks, last ? kMetaLast : 0);
                 uint8_t *st = ring + s * L::kStageBytes;
                 mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-#pragma unroll
-                for (int hf = 0; hf < L::kHalves; ++hf)
-                    tma_load_3d(st + hf * L::kRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
-#pragma unroll
-                for (int hf = 0; hf < L::kHalves; ++hf)
-                    tma_load_3d(st + L::kTileBytes + hf * L::kRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
+                // one box per tensor fills the tile's halves ([half][row][128 B])
+                tma_load_4d(st, &tm_k, &full[s], 0, sg.hk, row, 0, pol);
+                tma_load_4d(st + L::kTileBytes, &tm_v, &full[s], 0, sg.hk, row, 0, pol);
                 advance();
                 return true;
             };
@@ -251,6 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     const int k_cadd = mi >> 1;
     const int v_row = kbase + (mi >> 1) * 8 + (lane & 7);   // V^T: matrices (d lo/hi) x (keys lo/hi)
     const int v_cadd = mi & 1;
+    // tile layout: boxes of pb rows (64 packed; the page's keys, when pages
+    // are smaller, paged), each [half][row][128 B]: byte offset of row r's
+    // first half is (r / pb) * pb * D * 2 + (r % pb) * 128, the next half
+    // pb * 128 further; the 128-byte swizzle works on r mod 8 (pb >= 8)
+    const int pb = PAGED ? p.page_box : kBN;
+    const uint32_t half_stride = (uint32_t)pb * 128;
+    auto row_off = [&](int r) -> uint32_t {
+        return (uint32_t)((r / pb) * pb * L::kHalves * 128 + (r % pb) * 128);
+    };
+    const uint32_t k_ro = row_off(k_row), v_ro = row_off(v_row);
     float *ms = ored + kConsumerWarps * ROWS * OLD;           // [4][ROWS]
     float *lsum = ms + kConsumerWarps * ROWS;                  // [4][ROWS]
 
@@ -337,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 uint8_t *vt = ring + s * L::kStageBytes + L::kTileBytes;
                 for (int i = lane; i < (kbase + 16 - z0) * L::kHalves * 8; i += 32) {
                     const int r = z0 + i / (L::kHalves * 8), rest = i % (L::kHalves * 8);
-                    *reinterpret_cast<uint4 *>(vt + (rest >> 3) * L::kRegion + r * 128 + (rest & 7) * 16) =
+                    *reinterpret_cast<uint4 *>(vt + (rest >> 3) * half_stride + row_off(r) + (rest & 7) * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
                 zeroed = true;
@@ -352,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             for (int ks = 0; ks < KS; ++ks) {
                 const int hf = ks >> 2, c0 = (ks & 3) * 2;
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4(kst + hf * L::kRegion + swz(k_row, c0 + k_cadd), a0, a1, a2, a3);
+                ldsm_x4(kst + hf * half_stride + k_ro + (((c0 + k_cadd) ^ (k_row & 7)) << 4), a0, a1, a2, a3);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
             }
@@ -395,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             for (int mt = 0; mt < KS; ++mt) {
                 const int hf = mt >> 2, c0 = (mt & 3) * 2;
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4_trans(vst + hf * L::kRegion + swz(v_row, c0 + v_cadd), a0, a1, a2, a3);
+                ldsm_x4_trans(vst + hf * half_stride + v_ro + (((c0 + v_cadd) ^ (v_row & 7)) << 4), a0, a1, a2, a3);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
             }
