@@ -82,10 +82,11 @@ __device__ __forceinline__ int page_of(const Params &p, int b, int j) { return p
 
 // pull the block-table entries of keys [0, Lk) of sequence b into L2 (one
 // prefetch per 128-byte line), so the per-tile reads that follow hit there
-__device__ __forceinline__ void prefetch_pages(const Params &p, int b, int Lk) {
+// (the caller's lane `first` of `step` lanes takes every step-th line)
+__device__ __forceinline__ void prefetch_pages(const Params &p, int b, int Lk, int first = 0, int step = 1) {
     const int32_t *row = p.block_table + (long long)b * p.bt_stride;
     const int n = (Lk + (1 << p.page_shift) - 1) >> p.page_shift;
-    for (int i = 0; i < n; i += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + i));
+    for (int i = 32 * first; i < n; i += 32 * step) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + i));
 }
 
 constexpr int kMaxPageBoxes = 8;          // paged K/V: boxes per 64-key tile at the smallest page (8 keys)

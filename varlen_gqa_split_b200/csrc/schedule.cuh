@@ -310,7 +310,10 @@ __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int t
 // false, followed by none(seg): consumers finish their part of the unit at
 // that empty stage.  A callback returns false to stop the walk (a wait gave up);
 // the function then returns false.
-template <class Begin, class Tile, class None>
+// WARP: the whole warp calls it in step (every lane walks the same
+// schedule; lane 0 alone takes the claims and the result is broadcast), so
+// that the callbacks can spread their work over the lanes.
+template <bool WARP = false, class Begin, class Tile, class None>
 __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long long pb_first, long long lo,
                                            long long hi, Begin &&begin, Tile &&tile, None &&none) {
     OrderedWalker wk;
@@ -347,16 +350,24 @@ __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long lo
         // overlaps them; the tiles therefore cannot be told which one ends
         // the block's part, and an empty terminator stage (none) marks the
         // end instead.
+        // a claim's result lives on lane 0 until it is needed (WARP)
+        auto take = [&]() -> unsigned long long {
+            return (!WARP || (threadIdx.x & 31) == 0) ? atomicAdd(claim, inc) : 0ull;
+        };
+        auto seen = [&](unsigned long long v) -> unsigned long long {
+            if constexpr (WARP) return __shfl_sync(0xffffffffu, v, 0);
+            return v;
+        };
         int a_lo, a_hi;
-        range(atomicAdd(claim, inc), a_lo, a_hi);
+        range(seen(take()), a_lo, a_hi);
         while (a_lo < a_hi) {
             const bool more = up ? a_hi < ntiles : a_lo > 0;   // this range did not reach the far end
             unsigned long long pend = 0;
-            if (more) pend = atomicAdd(claim, inc);
+            if (more) pend = take();
             for (int i = 0; i < a_hi - a_lo; ++i)
                 if (!tile(seg, up ? a_lo + i : a_hi - 1 - i, false)) return false;
             if (!more) break;
-            range(pend, a_lo, a_hi);
+            range(seen(pend), a_lo, a_hi);
         }
         if (!none(seg)) return false;
     }

@@ -116,22 +116,25 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     __syncthreads();
 
     // ------------------------------------------------------------ producer
-    // One lane feeds the ring with the block's tiles (schedule.cuh
-    // feed_tiles).  Every stage carries its tile's key start and a flag in
-    // shared memory; the block's last stage of a unit is flagged (an empty
-    // stage carries the flag when the block got no tile of it).
+    // Feeds the ring with the block's tiles (schedule.cuh feed_tiles).  Every
+    // stage carries its tile's key start and a flag in shared memory; the
+    // block's last stage of a unit is flagged (an empty stage carries the
+    // flag when the block got no tile of it).  Packed: one lane.  Paged: the
+    // whole warp walks the schedule in step and each lane loads one box (a
+    // tile from small pages is up to 16 boxes), lane 0 doing the rest.
     if (warp == kConsumerWarps) {
-        if (lane == 0) {
+        if (PAGED || lane == 0) {
+            const unsigned wmask = PAGED ? 0xffffffffu : 1u;
+            const bool leader = lane == 0;
             const uint64_t pol = l2_evict_first();
             int s = 0, issued = 0;
             uint32_t phase = 0;
             // take the next free stage; false if the wait gave up
             auto acquire = [&]() -> bool {
-                if (issued >= stages && !mbar_wait(&empty[s], phase ^ 1)) {
-                    atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
-                    return false;
-                }
-                return true;
+                const bool w = issued < stages || mbar_wait(&empty[s], phase ^ 1);
+                if (__all_sync(wmask, w)) return true;
+                if (leader) atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
+                return false;
             };
             auto advance = [&]() {
                 ++issued;
@@ -140,71 +143,49 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                     phase ^= 1;
                 }
             };
+            // the stage's key start and flags, and the bytes its loads bring
+            // (before any lane issues one)
+            auto open_stage = [&](int ks, bool last) -> uint8_t * {
+                if (leader) {
+                    meta[s] = make_int2(ks, last ? kMetaLast : 0);
+                    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+                }
+                __syncwarp(wmask);
+                return ring + s * L::kStageBytes;
+            };
             auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
                 const int ks = tile * kBN;
-                if constexpr (PAGED) if (p.page_box == kBN && p.page_rows) {
-                    // paged, pages of 64 keys or more a whole number of rows apart: one
-                    // row index per tile, page * page_rows + slot, as lean as a packed
-                    // tile (the table read is issued before the stage wait)
-                    const int entry = page_entry(p, sg.b, ks);
-                    if (!acquire()) return false;
-                    const int row = page_checked(p, entry) * p.page_rows + (ks & ((1 << p.page_shift) - 1));
-                    meta[s] = make_int2(ks, last ? kMetaLast : 0);
-                    uint8_t *st = ring + s * L::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-                    tma_load_4d(st, &tm_k, &full[s], 0, sg.hk, row, 0, pol);          // all halves
-                    tma_load_4d(st + L::kTileBytes, &tm_v, &full[s], 0, sg.hk, row, 0, pol);
-                    advance();
-                    return true;
-                }
                 if constexpr (PAGED) {
-                    // paged, in general: the tile's keys in boxes of page_box keys,
-                    // each from its page; the table is read before the stage wait,
-                    // so the read overlaps it
-                    const int nbox = kBN / p.page_box;
-                    int pg[kMaxPageBoxes];
-                    uint32_t live = 0;                      // boxes holding keys of the sequence
-#pragma unroll
-                    for (int i = 0; i < kMaxPageBoxes; ++i) {
-                        if (i >= nbox) break;
-                        const int key = ks + i * p.page_box;
-                        pg[i] = 0;
-                        if (key < sg.s.Lk) {
-                            pg[i] = page_entry(p, sg.b, key);
-                            live |= 1u << i;
-                        }
-                    }
+                    // boxes of page_box keys, each from its page: lane i loads
+                    // box i / 2 of K (i even) or V (i odd); the table reads go
+                    // out before the stage wait, so they overlap it
+                    const int nbox = kBN / p.page_box, bi = lane >> 1;
+                    const bool mine = lane < 2 * nbox;
+                    const int key = ks + bi * p.page_box;
+                    const bool in = mine && key < sg.s.Lk;
+                    const int entry = in ? page_entry(p, sg.b, key) : 0;
                     if (!acquire()) return false;
-                    meta[s] = make_int2(ks, last ? kMetaLast : 0);
-                    uint8_t *st = ring + s * L::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-                    const int slot_mask = (1 << p.page_shift) - 1;
-#pragma unroll
-                    for (int i = 0; i < kMaxPageBoxes; ++i) {
-                        if (i >= nbox) break;
-                        // a box past the sequence (or a bad entry) reads page num_pages,
-                        // outside the map: zeros
-                        const int page = (live >> i) & 1u ? page_checked(p, pg[i]) : p.num_pages;
-                        const int slot = (ks + i * p.page_box) & slot_mask;   // 0 when pages are < 64 keys
-                        // box i holds its page_box rows of every half:
-                        // [half][row][128 B] at i * page_box * D * 2
-                        uint8_t *dk = st + i * p.page_box * L::kHalves * 128, *dv = dk + L::kTileBytes;
-                        if (p.page_rows) {
-                            tma_load_4d(dk, &tm_k, &full[s], 0, sg.hk, page * p.page_rows + slot, 0, pol);
-                            tma_load_4d(dv, &tm_v, &full[s], 0, sg.hk, page * p.page_rows + slot, 0, pol);
-                        } else {
-                            tma_load_5d(dk, &tm_k, &full[s], 0, sg.hk, slot, page, 0, pol);
-                            tma_load_5d(dv, &tm_v, &full[s], 0, sg.hk, slot, page, 0, pol);
-                        }
+                    uint8_t *st = open_stage(ks, last);
+                    if (mine) {
+                        // a box past the sequence (or a bad entry) reads page
+                        // num_pages, outside the map: zeros
+                        const int page = in ? page_checked(p, entry) : p.num_pages;
+                        const int slot = key & ((1 << p.page_shift) - 1);   // 0 when pages are < 64 keys
+                        // box bi holds its page_box rows of every half:
+                        // [half][row][128 B] at bi * page_box * D * 2
+                        uint8_t *dst = st + bi * p.page_box * L::kHalves * 128 + (lane & 1) * L::kTileBytes;
+                        const CUtensorMap *map = (lane & 1) ? &tm_v : &tm_k;
+                        if (p.page_rows)
+                            tma_load_4d(dst, map, &full[s], 0, sg.hk, page * p.page_rows + slot, 0, pol);
+                        else
+                            tma_load_5d(dst, map, &full[s], 0, sg.hk, slot, page, 0, pol);
                     }
                     advance();
                     return true;
                 }
                 if (!acquire()) return false;
                 const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
-                meta[s] = make_int2(ks, last ? kMetaLast : 0);
-                uint8_t *st = ring + s * L::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+                uint8_t *st = open_stage(ks, last);
                 // one box per tensor fills the tile's halves ([half][row][128 B])
                 tma_load_4d(st, &tm_k, &full[s], 0, sg.hk, row, 0, pol);
                 tma_load_4d(st + L::kTileBytes, &tm_v, &full[s], 0, sg.hk, row, 0, pol);
@@ -213,16 +194,18 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             };
             auto empty_stage = [&](const Segment &) -> bool {   // end of a unit without a tile
                 if (!acquire()) return false;
-                meta[s] = make_int2(0, kMetaLast | kMetaEmpty);
-                mbar_arrive(&full[s]);
+                if (leader) {
+                    meta[s] = make_int2(0, kMetaLast | kMetaEmpty);
+                    mbar_arrive(&full[s]);
+                }
                 advance();
                 return true;
             };
             auto begin = [&](const Segment &sg, int) -> bool {
-                if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk);
+                if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk, lane, 32);
                 return true;
             };
-            feed_tiles(p, b_first, pb_first, lo, hi, begin, load_tile, empty_stage);
+            feed_tiles<PAGED>(p, b_first, pb_first, lo, hi, begin, load_tile, empty_stage);
         }
         return;
     }
