@@ -177,13 +177,21 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const int G = p.G, QT = p.qtile;                         // query tokens per row tile
 
-    if (has_work && warp == kProducerWarp && lane == 0) {
+    if (has_work && warp == kProducerWarp && (PAGED || lane == 0)) {
         // ---------------------------------------------------------- producer
+        // packed: one lane; paged: the whole warp walks the schedule in step
+        // and each lane loads one box of a tile (up to 32 from small pages),
+        // lane 0 doing the rest
+        const unsigned wmask = PAGED ? 0xffffffffu : 1u;
+        const bool leader = lane == 0;
         const uint64_t pol = l2_evict_first();
         const uint32_t q_bytes = (uint32_t)(L::kHalves * G * QT * 128);
         int s = 0, issued = 0, k = 0;
         uint32_t phase = 0;
-        auto acquire = [&]() -> bool { return issued < stages || wait_bar(&empty[s], phase ^ 1, stop, p); };
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(wmask, wait_bar(bar, parity, stop, p));
+        };
+        auto acquire = [&]() -> bool { return issued < stages || wait_all(&empty[s], phase ^ 1); };
         auto advance = [&]() {
             ++issued;
             if (++s == stages) {
@@ -191,90 +199,65 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 phase ^= 1;
             }
         };
+        // the stage's key start and flags, and the bytes its loads bring
+        // (before any lane issues one)
+        auto open_stage = [&](int ks, bool last) -> uint8_t * {
+            if (leader) {
+                meta[s] = make_int2(ks, last ? kMetaLast : 0);
+                mbar_arrive_expect_tx(&full[s], L::kStage);
+            }
+            __syncwarp(wmask);
+            return ring + s * L::kStage;
+        };
         auto begin = [&](const Segment &sg, int) -> bool {
-            if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk);
+            if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk, lane, 32);
             const int qb = k & 1;
-            if (k >= 2 && !wait_bar(&q_free[qb], ((k - 2) >> 1) & 1, stop, p)) return false;
-            mbar_arrive_expect_tx(&q_full[qb], q_bytes);
-            // the box ends at the row tile's last query token
-            const int t_end = sg.s.q0 + sg.s.Lq - sg.rt * QT;
+            if (k >= 2 && !wait_all(&q_free[qb], ((k - 2) >> 1) & 1)) return false;
+            if (leader) {
+                mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+                // the box ends at the row tile's last query token
+                const int t_end = sg.s.q0 + sg.s.Lq - sg.rt * QT;
 #pragma unroll
-            for (int hf = 0; hf < L::kHalves; ++hf)
-                tma_load_3d(qbuf + qb * L::kQTile + hf * L::kQRegion, &tm_q, &q_full[qb], hf * 64, sg.hk * G,
-                            t_end - QT, pol);
+                for (int hf = 0; hf < L::kHalves; ++hf)
+                    tma_load_3d(qbuf + qb * L::kQTile + hf * L::kQRegion, &tm_q, &q_full[qb], hf * 64, sg.hk * G,
+                                t_end - QT, pol);
+            }
             ++k;
             return true;
         };
         auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
             const int ks = tile * kBN;
-            if constexpr (PAGED) if (p.page_box == kBN && p.page_rows) {
-                // paged, pages of 64 keys or more a whole number of rows apart: one
-                // row index per tile, page * page_rows + slot, as lean as a packed
-                // tile (the table read is issued before the stage wait)
-                const int entry = page_entry(p, sg.b, ks);
-                if (!acquire()) return false;
-                const int row = page_checked(p, entry) * p.page_rows + (ks & ((1 << p.page_shift) - 1));
-                meta[s] = make_int2(ks, last ? kMetaLast : 0);
-                uint8_t *st = ring + s * L::kStage;
-                mbar_arrive_expect_tx(&full[s], L::kStage);
-#pragma unroll
-                for (int hf = 0; hf < L::kHalves; ++hf)
-                    tma_load_3d(st + hf * L::kKvRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
-#pragma unroll
-                for (int hf = 0; hf < L::kHalves; ++hf)
-                    tma_load_3d(st + L::kKvTile + hf * L::kKvRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
-                advance();
-                return true;
-            }
             if constexpr (PAGED) {
-                // paged, in general: the tile's keys in boxes of page_box keys,
-                // each from its page; the table is read before the stage wait,
-                // so the read overlaps it
-                const int nbox = kBN / p.page_box;
-                int pg[kMaxPageBoxes];
-                uint32_t live = 0;                      // boxes holding keys of the sequence
-#pragma unroll
-                for (int i = 0; i < kMaxPageBoxes; ++i) {
-                    if (i >= nbox) break;
-                    const int key = ks + i * p.page_box;
-                    pg[i] = 0;
-                    if (key < sg.s.Lk) {
-                        pg[i] = page_entry(p, sg.b, key);
-                        live |= 1u << i;
-                    }
-                }
+                // boxes of page_box keys x one D-half, each from its page:
+                // lane l loads box l / (2 halves) of K or V; the table reads
+                // go out before the stage wait, so they overlap it
+                constexpr int kPer = 2 * L::kHalves;                // loads per box of keys
+                const int nbox = kBN / p.page_box, bi = lane / kPer, rem = lane % kPer;
+                const int tv = rem / L::kHalves, hf = rem % L::kHalves;
+                const bool mine = lane < nbox * kPer;
+                const int key = ks + bi * p.page_box;
+                const bool in = mine && key < sg.s.Lk;
+                const int entry = in ? page_entry(p, sg.b, key) : 0;
                 if (!acquire()) return false;
-                meta[s] = make_int2(ks, last ? kMetaLast : 0);
-                uint8_t *st = ring + s * L::kStage;
-                mbar_arrive_expect_tx(&full[s], L::kStage);
-                const int slot_mask = (1 << p.page_shift) - 1;
-#pragma unroll
-                for (int i = 0; i < kMaxPageBoxes; ++i) {
-                    if (i >= nbox) break;
-                    // a box past the sequence (or a bad entry) reads page num_pages,
-                    // outside the map: zeros
-                    const int page = (live >> i) & 1u ? page_checked(p, pg[i]) : p.num_pages;
-                    const int slot = (ks + i * p.page_box) & slot_mask;   // 0 when pages are < 64 keys
-#pragma unroll
-                    for (int hf = 0; hf < L::kHalves; ++hf) {
-                        uint8_t *dk = st + hf * L::kKvRegion + i * p.page_box * 128, *dv = dk + L::kKvTile;
-                        if (p.page_rows) {
-                            tma_load_3d(dk, &tm_k, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
-                            tma_load_3d(dv, &tm_v, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
-                        } else {
-                            tma_load_4d(dk, &tm_k, &full[s], hf * 64, sg.hk, slot, page, pol);
-                            tma_load_4d(dv, &tm_v, &full[s], hf * 64, sg.hk, slot, page, pol);
-                        }
-                    }
+                uint8_t *st = open_stage(ks, last);
+                if (mine) {
+                    // a box past the sequence (or a bad entry) reads page
+                    // num_pages, outside the map: zeros
+                    const int page = in ? page_checked(p, entry) : p.num_pages;
+                    const int slot = key & ((1 << p.page_shift) - 1);       // 0 when pages are < 64 keys
+                    uint8_t *dst = st + tv * L::kKvTile + hf * L::kKvRegion + bi * p.page_box * 128;
+                    const CUtensorMap *map = tv ? &tm_v : &tm_k;
+                    if (p.page_rows)
+                        tma_load_3d(dst, map, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
+                    else
+                        tma_load_4d(dst, map, &full[s], hf * 64, sg.hk, slot, page, pol);
                 }
                 advance();
                 return true;
             }
             if (!acquire()) return false;
             const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
-            meta[s] = make_int2(ks, last ? kMetaLast : 0);
-            uint8_t *st = ring + s * L::kStage;
-            mbar_arrive_expect_tx(&full[s], L::kStage);
+            uint8_t *st = open_stage(ks, last);
 #pragma unroll
             for (int hf = 0; hf < L::kHalves; ++hf)
                 tma_load_3d(st + hf * L::kKvRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
@@ -286,12 +269,14 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         };
         auto empty_stage = [&](const Segment &) -> bool {
             if (!acquire()) return false;
-            meta[s] = make_int2(0, kMetaLast | kMetaEmpty);
-            mbar_arrive(&full[s]);
+            if (leader) {
+                meta[s] = make_int2(0, kMetaLast | kMetaEmpty);
+                mbar_arrive(&full[s]);
+            }
             advance();
             return true;
         };
-        if (!feed_tiles(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage)) *stop = 1;
+        if (!feed_tiles<PAGED>(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage)) *stop = 1;
         // let the loads in flight land before the block can exit (bounded,
         // also after a stop: the copies target this block's shared memory)
         for (int i = 0; i < min(issued, stages); ++i) {
