@@ -119,12 +119,13 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     // Feeds the ring with the block's tiles (schedule.cuh feed_tiles).  Every
     // stage carries its tile's key start and a flag in shared memory; the
     // block's last stage of a unit is flagged (an empty stage carries the
-    // flag when the block got no tile of it).  Packed: one lane.  Paged: the
-    // whole warp walks the schedule in step and each lane loads one box (a
-    // tile from small pages is up to 16 boxes), lane 0 doing the rest.
+    // flag when the block got no tile of it).  The whole warp walks the
+    // schedule in step and each lane loads one box (K or V of a tile, or of
+    // a page's keys: a tile from small pages is up to 16 boxes), lane 0
+    // doing the rest.
     if (warp == kConsumerWarps) {
-        if (PAGED || lane == 0) {
-            const unsigned wmask = PAGED ? 0xffffffffu : 1u;
+        {
+            const unsigned wmask = 0xffffffffu;
             const bool leader = lane == 0;
             const uint64_t pol = l2_evict_first();
             int s = 0, issued = 0;
@@ -187,8 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
                 uint8_t *st = open_stage(ks, last);
                 // one box per tensor fills the tile's halves ([half][row][128 B])
-                tma_load_4d(st, &tm_k, &full[s], 0, sg.hk, row, 0, pol);
-                tma_load_4d(st + L::kTileBytes, &tm_v, &full[s], 0, sg.hk, row, 0, pol);
+                if (lane < 2)
+                    tma_load_4d(st + lane * L::kTileBytes, lane ? &tm_v : &tm_k, &full[s], 0, sg.hk, row, 0, pol);
                 advance();
                 return true;
             };
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
                 if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk, lane, 32);
                 return true;
             };
-            feed_tiles<PAGED>(p, b_first, pb_first, lo, hi, begin, load_tile, empty_stage);
+            feed_tiles<true>(p, b_first, pb_first, lo, hi, begin, load_tile, empty_stage);
         }
         return;
     }

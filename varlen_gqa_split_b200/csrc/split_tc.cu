@@ -177,12 +177,12 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const int G = p.G, QT = p.qtile;                         // query tokens per row tile
 
-    if (has_work && warp == kProducerWarp && (PAGED || lane == 0)) {
+    if (has_work && warp == kProducerWarp) {
         // ---------------------------------------------------------- producer
-        // packed: one lane; paged: the whole warp walks the schedule in step
-        // and each lane loads one box of a tile (up to 32 from small pages),
-        // lane 0 doing the rest
-        const unsigned wmask = PAGED ? 0xffffffffu : 1u;
+        // the whole warp walks the schedule in step and each lane loads one
+        // box of a tile (a D-half of K or V; up to 32 boxes from small
+        // pages), lane 0 doing the rest
+        const unsigned wmask = 0xffffffffu;
         const bool leader = lane == 0;
         const uint64_t pol = l2_evict_first();
         const uint32_t q_bytes = (uint32_t)(L::kHalves * G * QT * 128);
@@ -258,12 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             if (!acquire()) return false;
             const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
             uint8_t *st = open_stage(ks, last);
-#pragma unroll
-            for (int hf = 0; hf < L::kHalves; ++hf)
-                tma_load_3d(st + hf * L::kKvRegion, &tm_k, &full[s], hf * 64, sg.hk, row, pol);
-#pragma unroll
-            for (int hf = 0; hf < L::kHalves; ++hf)
-                tma_load_3d(st + L::kKvTile + hf * L::kKvRegion, &tm_v, &full[s], hf * 64, sg.hk, row, pol);
+            if (lane < 2 * L::kHalves) {                        // lane: (K or V, D-half)
+                const int tv = lane / L::kHalves, hf = lane % L::kHalves;
+                tma_load_3d(st + tv * L::kKvTile + hf * L::kKvRegion, tv ? &tm_v : &tm_k, &full[s], hf * 64, sg.hk,
+                            row, pol);
+            }
             advance();
             return true;
         };
@@ -276,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             advance();
             return true;
         };
-        if (!feed_tiles<PAGED>(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage)) *stop = 1;
+        if (!feed_tiles<true>(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage)) *stop = 1;
         // let the loads in flight land before the block can exit (bounded,
         // also after a stop: the copies target this block's shared memory)
         for (int i = 0; i < min(issued, stages); ++i) {
