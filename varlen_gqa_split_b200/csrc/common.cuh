@@ -38,12 +38,15 @@ __device__ __forceinline__ int live_chunks(int Lk, int chunk) {
 // Reads the lengths of sequence b and checks them against the plan.  Returns
 // false (and, when `report`, records the reason) if the sequence must be
 // skipped.  The same test runs in every kernel that touches the sequence.
+// spec: a speculative read made before the kernel has waited for the one it
+// depends on (the value may still change); it goes to L2 only, so that no
+// line of cu_seqlens stays in L1 for the later, real reads to hit.
 __device__ __forceinline__ bool load_lengths(const Params &p, int b, bool report,
-                                             int &q0, int &Lq, int &k0, int &Lk) {
-    q0 = __ldg(p.cu_q + b);
-    const int q1 = __ldg(p.cu_q + b + 1);
-    k0 = __ldg(p.cu_k + b);
-    const int k1 = __ldg(p.cu_k + b + 1);
+                                             int &q0, int &Lq, int &k0, int &Lk, bool spec = false) {
+    q0 = spec ? __ldcg(p.cu_q + b) : __ldg(p.cu_q + b);
+    const int q1 = spec ? __ldcg(p.cu_q + b + 1) : __ldg(p.cu_q + b + 1);
+    k0 = spec ? __ldcg(p.cu_k + b) : __ldg(p.cu_k + b);
+    const int k1 = spec ? __ldcg(p.cu_k + b + 1) : __ldg(p.cu_k + b + 1);
     Lq = q1 - q0;
     Lk = k1 - k0;
     uint32_t bad = 0;
@@ -185,6 +188,21 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
         "l"(policy)
         : "memory");
+}
+
+// L2 prefetch of a tile (no shared memory, no barrier): a hint, and safe at
+// any coordinates, since the tensor map bounds what it may touch
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tma_load_5d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,

@@ -30,6 +30,10 @@ namespace sched {
 
 constexpr int kBN = 64;                   // keys per tile
 constexpr int kClaim = 2;                 // tiles per claim on a shared unit's counter
+// K/V bytes per block prefetched into L2 before the dependency wait
+// (first_tiles; 37 MB over 148 blocks, about what the DRAM delivers while a
+// back-to-back predecessor drains: 128 KB gained less, 512 KB lost it all)
+constexpr int kPrefetchBytes = 256 * 1024;
 
 struct SeqLen {
     int q0, Lq, k0, Lk;
@@ -50,9 +54,9 @@ __device__ __forceinline__ int rt_tiles(const SeqLen &s, int rt, int qtile) {
 // tiles.  A unit's real tile t sits at position unit_cost + t of its range.
 __device__ __forceinline__ int unit_weight(const Params &p, int tiles) { return max(tiles, 1) + p.unit_cost; }
 
-__device__ __forceinline__ SeqLen seq_len(const Params &p, int b, bool report) {
+__device__ __forceinline__ SeqLen seq_len(const Params &p, int b, bool report, bool spec = false) {
     SeqLen s;
-    const bool ok = load_lengths(p, b, report, s.q0, s.Lq, s.k0, s.Lk);
+    const bool ok = load_lengths(p, b, report, s.q0, s.Lq, s.k0, s.Lk, spec);
     if (!ok || s.Lq <= 0) {
         s.nrt = s.tpu = 0;
     } else if (s.Lq <= p.qtile) {                 // one row tile: every decode sequence
@@ -95,15 +99,18 @@ struct SegWalker {
     int nt, w;            // the current unit's tiles and weight
     long long Pu;         // global index of the current unit's first position
     long long g, hi;
+    bool spec;            // speculative reads of cu_seqlens (load_lengths)
 
     __device__ void set_unit(const Params &p) {
         nt = rt_tiles(s, rt, p.qtile);
         w = unit_weight(p, nt);
     }
 
-    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi_) {
+    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi_,
+                         bool spec_ = false) {
+        spec = spec_;
         b = b_first;
-        s = seq_len(p, b, false);
+        s = seq_len(p, b, false, spec);
         hk = (int)((lo - pb_first) / s.tpu);
         Pu = pb_first + (long long)hk * s.tpu;
         rt = 0;
@@ -146,7 +153,7 @@ struct SegWalker {
                             g = hi;
                             break;
                         }
-                        s = seq_len(p, b, false);
+                        s = seq_len(p, b, false, spec);
                     } while (s.tpu == 0);
                 }
             }
@@ -168,8 +175,9 @@ struct OrderedWalker {
     bool has_first, has_last;
     int phase;            // 0: inside units, 1: the start-cut unit, 2: the end-cut unit, 3: done
 
-    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi) {
-        wk.init(p, b_first, pb_first, lo, hi);
+    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi,
+                         bool spec = false) {
+        wk.init(p, b_first, pb_first, lo, hi, spec);
         wk_lo = lo;
         has_first = has_last = false;
         phase = 0;
@@ -244,12 +252,12 @@ struct Share {
 
 // scan: nthreads / 32 long long of shared memory (one per warp); first: 3.
 __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int tid, int nthreads, bool report,
-                                            long long *scan, long long *first, Share &sh) {
+                                            long long *scan, long long *first, Share &sh, bool spec = false) {
     const int warp = tid >> 5, lane = tid & 31;
     const int per = (p.B_max + nthreads - 1) / nthreads;
     const int b_lo = min(p.B_max, tid * per), b_hi = min(p.B_max, b_lo + per);
     long long my = 0;
-    for (int b = b_lo; b < b_hi; ++b) my += (long long)p.Hkv * seq_len(p, b, report).tpu;
+    for (int b = b_lo; b < b_hi; ++b) my += (long long)p.Hkv * seq_len(p, b, report, spec).tpu;
     long long incl = my;                                    // warp-inclusive scan
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -280,7 +288,7 @@ __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int t
     long long pb = my_start;
     if (sh.lo >= pb && sh.lo < pb + my) {
         for (int b = b_lo; b < b_hi; ++b) {
-            const long long w = (long long)p.Hkv * seq_len(p, b, false).tpu;
+            const long long w = (long long)p.Hkv * seq_len(p, b, false, spec).tpu;
             if (sh.lo < pb + w) {
                 first[0] = b;
                 first[1] = pb;
@@ -372,6 +380,51 @@ __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long lo
         if (!none(seg)) return false;
     }
     return true;
+}
+
+// For a speculative L2 prefetch before the kernel's dependency wait: the
+// first `budget` tiles the block is likely to load, fn(seg, t) for each,
+// spread over the calling warp's lanes (lane i takes tiles i, i + 32, ...) --
+// but only for a block whose share holds no whole unit, that is one that
+// starts on a unit shared with other blocks (few, long units: long-context
+// decode, short-query batches).  A block that starts on units of its own
+// prefetches nothing: measured on continuous batching, such prefetches
+// slowed the calls by about 1.5%, the previous call's last blocks, which
+// wait on DRAM latency, getting slower under the added traffic.
+// In the static mode a cut unit starts where feed_tiles starts it.  In the
+// run-time balanced mode the block holding the unit's front starts at its
+// tile 0; the others claim from the back, and together their first claims
+// take the unit's last tiles, so the j-th of them (j >= 1 in share order)
+// takes tiles [nt - j * budget, nt - (j - 1) * budget).
+template <class Fn>
+__device__ __forceinline__ void first_tiles(const Params &p, int c, const Share &sh, int budget, bool spec,
+                                            Fn &&fn) {
+    OrderedWalker wk;
+    wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, spec);
+    Segment seg;
+    int role;
+    const int lane = threadIdx.x & 31;
+    int done = 0;
+    while (done < budget && wk.next(p, seg, role)) {
+        if (role == 0) return;                         // whole units come first: the share has one
+        const int nt = seg.nt;
+        int a = 0, dir = 1, cnt;
+        if (!p.dynamic) {
+            a = max(0, seg.t0 - p.unit_cost);
+            cnt = min(nt, max(0, seg.t1 - p.unit_cost)) - a;
+        } else if (seg.t0 == 0) {
+            cnt = nt;
+        } else {
+            const int j = c - block_of(seg.Pu, sh.T, sh.Ce);
+            const int e = nt - (j - 1) * budget;
+            a = e - 1;
+            dir = -1;
+            cnt = min(e, budget);
+        }
+        cnt = max(0, min(cnt, budget - done));
+        for (int i = lane; i < cnt; i += 32) fn(seg, a + dir * i);
+        done += cnt;
+    }
 }
 
 }  // namespace sched

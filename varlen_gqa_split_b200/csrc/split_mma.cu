@@ -99,11 +99,28 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
         prefetch_tensormap(&tm_v);
     }
     // Launched as a programmatic dependent, the block may start while the
-    // previous kernel in the stream still runs; everything above touches only
-    // this block's shared memory.  Wait for that kernel (it may write the
-    // inputs, and a previous call's combine resets the counters used below)
-    // before reading any global memory.  Only then may this call's combine
-    // kernel launch: it relies on the counters being reset.
+    // previous kernel in the stream still runs, which leaves the DRAM idle as
+    // it ends.  Meanwhile the block computes a speculative schedule from
+    // cu_seqlens as they read now (L2-only reads, so no stale line stays in
+    // L1) and, if its share starts on a unit shared with other blocks,
+    // prefetches its first tiles into L2 (schedule.cuh first_tiles).  Both
+    // are hints: the L2 is coherent, so a prefetched line never hides a later
+    // write, and the tensor map bounds every prefetch whatever the lengths
+    // read.
+    if constexpr (!PAGED) {
+        Share sp;
+        if (block_share(p, c, gridDim.x, tid, kThreads, false, scan, first, sp, true) && warp == kConsumerWarps)
+            first_tiles(p, c, sp, kPrefetchBytes / L::kStageBytes, true, [&](const Segment &sg, int t) {
+                const int row = sg.s.k0 + min(t * kBN, sg.s.Lk - kBN);
+                tma_prefetch_4d(&tm_k, 0, sg.hk, row, 0);
+                tma_prefetch_4d(&tm_v, 0, sg.hk, row, 0);
+            });
+        __syncthreads();   // scan / first are reused below
+    }
+    // Wait for that kernel (it may write the inputs, and a previous call's
+    // combine resets the counters used below) before any read that counts.
+    // Only then may this call's combine kernel launch: it relies on the
+    // counters being reset.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 

@@ -163,9 +163,24 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         tc::tmem_relinquish();
     }
     // Launched as a programmatic dependent, the block may start while the
-    // previous kernel in the stream still runs; everything above touches only
-    // this block's shared and tensor memory.  Wait for that kernel before
-    // reading global memory; only then may this call's combine kernel launch.
+    // previous kernel in the stream still runs.  Meanwhile it prefetches its
+    // first K/V tiles into L2 under a speculative schedule (the warp-MMA
+    // kernel does the same; both are hints that no later write can make
+    // stale).  Then it waits for that kernel before the reads that count;
+    // only then may this call's combine kernel launch.
+    if constexpr (!PAGED) {
+        Share sp;
+        if (block_share(p, c, gridDim.x, tid, kThreads, false, scan, first, sp, true) && warp == kProducerWarp)
+            first_tiles(p, c, sp, kPrefetchBytes / L::kStage, true, [&](const Segment &sg, int t) {
+                const int row = sg.s.k0 + min(t * kBN, sg.s.Lk - kBN);
+#pragma unroll
+                for (int hf = 0; hf < L::kHalves; ++hf) {
+                    tma_prefetch_3d(&tm_k, hf * 64, sg.hk, row);
+                    tma_prefetch_3d(&tm_v, hf * 64, sg.hk, row);
+                }
+            });
+        __syncthreads();   // scan / first are reused below
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
