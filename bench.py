@@ -374,7 +374,8 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[0], sh.Hq, dtype=torch.float32, device=dev)
     plan = Plan(sh.B, sh.s_max, sh.Hq, sh.Hkv, sh.D, sh.max_q, nsplit=args.nsplit, variant=args.variant,
-                stages=args.stages, combine=args.combine, ctas=args.ctas)
+                stages=args.stages, combine=args.combine, ctas=args.ctas,
+                deterministic=int(args.deterministic))
     info = plan.info
     launches_per_call = 2 if info["combine"] == 1 else 1     # split (+ combine kernel)
 
@@ -613,6 +614,8 @@ def main():
     ap.add_argument("--stages", type=int, default=0)
     ap.add_argument("--combine", type=int, default=0)
     ap.add_argument("--ctas", type=int, default=0)
+    ap.add_argument("--deterministic", action="store_true",
+                    help="static shares, bitwise repeatable (no run-time claims)")
     ap.add_argument("--page-size", type=int, default=0,
                     help="read K/V from a paged cache with pages of this many tokens (0: packed)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

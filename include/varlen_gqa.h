@@ -94,8 +94,11 @@ typedef struct {
     int combine;   /* ATTN_COMBINE_*                                            */
     int ctas;      /* tensor-core path: blocks sharing the tile space; >= 1     */
     int deterministic; /* 1: bitwise-repeatable results (static tile shares);
-                          0: blocks that share a unit balance it between them
-                          at run time, results equal within rounding           */
+                          -1: blocks that share a unit balance it between them
+                          at run time, results equal within rounding;
+                          0: the plan's choice: run-time balancing on the
+                          warp-MMA path, static shares on the tcgen05 path
+                          (the CUDA-core path is always repeatable)           */
 } attn_overrides;
 
 /* What the planner chose (attn_plan_info). */

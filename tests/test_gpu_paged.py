@@ -89,7 +89,7 @@ def test_paged_split_units_and_block_counts(variant):
     batch = W.make_batch(sh, [1, max_q, min(2, max_q)], [9000, 4097, 3001], seed=41, gen_device="cuda")
     pc = W.paginate(batch.k, batch.v, batch.cu_k, sh.B, 16, sh.s_max, seed=5)
     ref_o, ref_l = oracle_full(batch)
-    for kw in ({"ctas": 7}, {"ctas": 7, "deterministic": 1}, {}):
+    for kw in ({"ctas": 7}, {"ctas": 7, "deterministic": 1}, {"ctas": 7, "deterministic": -1}, {}):
         plan = plan_for(sh, variant=variant, **kw)
         out, lse = _run_paged(plan, batch, pc)
         assert plan.check_error() == 0

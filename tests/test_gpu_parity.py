@@ -140,7 +140,7 @@ def test_block_count_invariance_mma(stages, det):
         assert np.abs(o - outs[0]).max() <= 2 * ATOL_OUT
 
 
-@pytest.mark.parametrize("stages,det", [(0, 0), (0, 1), (2, 0), (3, 1)])
+@pytest.mark.parametrize("stages,det", [(0, -1), (0, 1), (2, -1), (3, 0)])
 def test_block_count_invariance_tc(stages, det):
     """The tcgen05 path at 1 .. 2 x SM-count blocks on a short-query batch:
     whole units, units cut into many parts, a unit without keys, and rows
@@ -193,7 +193,7 @@ def test_variants_agree():
     assert np.abs(l1[fin] - l2[fin]).max() <= 2 * ATOL_LSE
 
 
-@pytest.mark.parametrize("kw", [{"deterministic": 1}, {"variant": TC, "deterministic": 1},
+@pytest.mark.parametrize("kw", [{"deterministic": 1}, {"variant": TC, "deterministic": 1}, {"variant": TC},
                                 {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_FUSED},
                                 {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_KERNEL}])
 def test_repeat_runs_bitwise_equal(kw):
@@ -213,7 +213,7 @@ def test_dynamic_balance_repeats_within_rounding():
     # other and with the oracle within the tolerance, not bit for bit
     batch = W.workload("long", gen_device="cuda")
     plan = plan_for(batch.shape)
-    assert plan.info["deterministic"] == 0
+    assert plan.info["deterministic"] == 0 and plan.info["variant"] == MMA
     ref_o, ref_l = oracle_full(batch)
     cov = covered_rows(batch)
     runs = [run_gpu(plan, batch) for _ in range(4)]
@@ -314,7 +314,9 @@ def test_exhaustive_small_lengths_placement(variant):
                                 {"variant": MMA, "ctas": 64}, {"variant": MMA},
                                 {"variant": MMA, "ctas": 64, "deterministic": 1},
                                 {"variant": TC, "ctas": 1}, {"variant": TC, "ctas": 5}, {"variant": TC},
-                                {"variant": TC, "ctas": 64, "deterministic": 1}])
+                                {"variant": TC, "ctas": 64, "deterministic": 1},
+                                {"variant": TC, "ctas": 5, "deterministic": -1},
+                                {"variant": TC, "ctas": 64, "deterministic": -1}])
 def test_ragged_multi_tile_placement(kw):
     """Lengths spanning several 64-key tiles, units cut across blocks, short
     sequences whose tile starts before the buffer (negative TMA
@@ -449,7 +451,7 @@ def test_tc_row_tiles_long_queries(Hq, Hkv, D, max_q):
     batch = W.make_batch(sh, lq, lk, seed=29, gen_device="cuda")
     ref_o, ref_l = oracle_full(batch)
     cov = covered_rows(batch)
-    for kw in ({}, {"ctas": 5}, {"ctas": 5, "deterministic": 1}):
+    for kw in ({}, {"ctas": 5}, {"ctas": 5, "deterministic": 1}, {"ctas": 5, "deterministic": -1}):
         plan = plan_for(sh, **kw)
         assert plan.info["variant"] == TC, plan.info
         out, lse = run_gpu(plan, batch, extra_q_rows=2)

@@ -139,7 +139,8 @@ class Plan:
 
     Plan(B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
     stages=0, combine=0, ctas=0, deterministic=0) -- the keyword choices
-    override the planner (0 = its own)."""
+    override the planner (0 = its own; deterministic=1 asks for static tile
+    shares, -1 for run-time balancing of shared units)."""
 
     def __init__(self, B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
                  stages=0, combine=0, ctas=0, deterministic=0):

@@ -265,7 +265,13 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         d.grid_x = d.ctas;
         d.grid_y = 1;
         d.grid_z = 1;
-        d.deterministic = o && o->deterministic ? 1 : 0;
+        // static shares unless asked otherwise on the tensor-core path (its
+        // run-time claims measured slower: short-query batches 56.0 -> 53.8 us,
+        // 16-key pages 64.1 -> 52.6 us, prefill equal), run-time claims on the
+        // warp-MMA decode path (long-context 28.6 -> 27.5 us, ragged
+        // 183 -> 175 us); the override's sign picks either
+        const int det_req = o ? o->deterministic : 0;
+        d.deterministic = det_req > 0 ? 1 : det_req < 0 ? 0 : (tcv ? 1 : 0);
         d.combine = ATTN_COMBINE_KERNEL;     // slot-parallel combine, programmatic dependent launch
         d.combine_blocks = 2 * d.ctas * combine_slots_split((Hq / Hkv) * qtile, D);
         n_ticket = 3 * (size_t)B_max * Hkv * max_rt;   // per unit: tile claims (64-bit), part count
