@@ -172,13 +172,42 @@ def measured_tensor_peak():
         return 1590.0, "fallback 1.59 PFLOP/s (pool measurement)"
 
 
+def strip_c_comments(src: str) -> str:
+    """The source with // and /* */ comments removed (string and character
+    literals kept as they are), trailing blanks cut and blank lines dropped:
+    what the compiler sees, up to layout."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (l.rstrip() for l in "".join(out).split("\n"))
+    return "\n".join(l for l in lines if l)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the library's C++/CUDA sources without their comments, so that
+    a recorded ncu capture stays attached to the code it measured and a
+    comment edit does not detach it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "varlen_gqa_split_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h", ".cpp")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + strip_c_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

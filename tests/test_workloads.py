@@ -133,3 +133,13 @@ def test_recorded_traffic_follows_the_source_hash():
             assert got is None and "changed" in note
     assert bench.recorded_traffic("long", "another_kernel")[0] is None
     assert bench.recorded_traffic("no_such_workload", "split_mma_kernel")[0] is None
+
+
+def test_comment_edits_keep_the_source_hash():
+    import bench
+    a = 'int f(int x) {\n    return x + 1;   // one more\n}\n'
+    b = '/* f: the successor */\nint f(int x) {\n\n    return x + 1;\n}\n'
+    c = 'int f(int x) {\n    return x + 2;\n}\n'
+    assert bench.strip_c_comments(a) == bench.strip_c_comments(b) != bench.strip_c_comments(c)
+    s = 'const char *p = "a // b /* c */"; char q = \'"\';  // tail'
+    assert bench.strip_c_comments(s) == 'const char *p = "a // b /* c */"; char q = \'"\';'
