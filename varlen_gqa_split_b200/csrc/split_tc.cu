@@ -4,16 +4,19 @@
 // longer queries as several row tiles of the sequence, each its own unit.
 //
 // Same schedule as the warp-MMA kernel (schedule.cuh: equal shares of the
-// flattened 64-key tiles, cut units merged by the slot combine kernel), but
+// flattened 64-key tiles, cut units merged by the slot combine kernel; by
+// default the shares stay static on this path, without run-time claims), but
 // the G query heads times the q_len query tokens of a unit form the M = 128
 // side of real tensor-core tiles (kernbench2 docs/adr-proposed commit log,
 // GQA entry: G folded into the matmul M dimension; every K/V byte is read
 // once per KV head):
 //     S [128 rows x 64 keys]  = Q [128 x D] . K^T            (tcgen05.mma, S in tensor memory)
-//     O [128 rows x D]       += P [128 x 64 keys] . V        (P bf16 in shared memory, O in tensor memory)
+//     O [128 rows x D]       += P [128 x 64 keys] . V        (P bf16 and O in tensor memory)
 //
 // Warp roles (320 threads):
-//   warp 9, one lane -- producer: loads each unit's Q tile (one TMA box of G
+//   warp 9 -- producer (the whole warp walks the schedule in step, each lane
+//     issuing one box, lane 0 taking claims and stage bookkeeping): loads each
+//     unit's Q tile (one TMA box of G
 //     heads x qtile tokens, right-aligned so it ends at the row tile's last
 //     query token; rows past the sequence's own tokens are never written)
 //     into one of two Q buffers, then streams the unit's K and V tiles into a
