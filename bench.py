@@ -17,6 +17,14 @@ over the actual ragged lengths plus Q and O (lse is reported apart).  With N > 1
 sequences: weak scaling, no collective on the data path) and the time is the
 max over ranks.
 
+The timed pass of K calls is repeated (the same number of passes on every
+rank, about a quarter of a second of device time in all) and the median pass
+gives the value; the spread of the passes and the SM clock sampled throughout
+are reported beside it.  Unless --only is given, a one-GPU run also measures
+the method's other workloads (ragged, continuous batching over all 100 length
+draws, short query, tiny) in the same process and reports them under
+"workloads", each with its CPU baseline.
+
 --impl reference times the fp64 CPU oracle on the host cores instead (rank 0
 only), on a bounded sample of the same workload per step.
 
@@ -320,29 +328,39 @@ def run_reference(args, batch: W.Batch) -> dict:
     }
 
 
-def cpu_baseline(batch: W.Batch, bytes_: dict, budget_s: float = 20.0) -> dict:
-    """The oracle as it stands on the host cores, on a bounded sample of the
-    same workload, scaled to GB/s of the workload's algorithmic bytes."""
+def cpu_baseline(batch: W.Batch, bytes_: dict, budget_s: float = 20.0, threads: int | None = None,
+                 seed: int = 1) -> dict:
+    """The oracle as it stands on the host cores (all of them, or `threads`),
+    on a bounded sample of the same workload, scaled to GB/s of the
+    workload's algorithmic bytes."""
     import oracle
     sh = batch.shape
-    qb, kb, vb = W.bits(batch.q), W.bits(batch.k), W.bits(batch.v)
-    lens_q, lens_k = batch.lens_q, batch.lens_k
-    rows_all = np.array([(b, qi, h) for b in range(len(lens_q)) for qi in range(int(lens_q[b]))
-                         for h in range(sh.Hq)], dtype=np.int64)
-    # work per row ~ its visible keys; sample whole rows until the budget is met
-    t0 = time.perf_counter()
-    oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, rows_all[:8], B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv,
-                          D=sh.D, causal=sh.causal)
-    t8 = max(time.perf_counter() - t0, 1e-4)
-    n = int(min(len(rows_all), max(8, 8 * (budget_s / 3) / t8)))
-    rng = np.random.default_rng(1)
-    sel = rows_all if n >= len(rows_all) else rows_all[np.sort(rng.choice(len(rows_all), n, replace=False))]
-    ts = []
-    for _ in range(3):
+    all_threads = oracle.num_threads()
+    if threads:
+        oracle.set_num_threads(threads)
+    try:
+        qb, kb, vb = W.bits(batch.q), W.bits(batch.k), W.bits(batch.v)
+        lens_q, lens_k = batch.lens_q, batch.lens_k
+        rows_all = np.array([(b, qi, h) for b in range(len(lens_q)) for qi in range(int(lens_q[b]))
+                             for h in range(sh.Hq)], dtype=np.int64)
+        # work per row ~ its visible keys; sample whole rows until the budget is met
         t0 = time.perf_counter()
-        oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, sel, B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv,
+        oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, rows_all[:8], B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv,
                               D=sh.D, causal=sh.causal)
-        ts.append(time.perf_counter() - t0)
+        t8 = max(time.perf_counter() - t0, 1e-4)
+        n = int(min(len(rows_all), max(8, 8 * (budget_s / 3) / t8)))
+        rng = np.random.default_rng(seed)
+        sel = rows_all if n >= len(rows_all) else rows_all[np.sort(rng.choice(len(rows_all), n, replace=False))]
+        ts = []
+        for _ in range(3):
+            t0 = time.perf_counter()
+            oracle.attention_rows(qb, kb, vb, batch.cu_q, batch.cu_k, sel, B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv,
+                                  D=sh.D, causal=sh.causal)
+            ts.append(time.perf_counter() - t0)
+        cores = oracle.num_threads()
+    finally:
+        if threads:
+            oracle.set_num_threads(all_threads)
     t = statistics.median(ts)
     # scale: the sample's share of the workload's (row x key) work
     vis = lambda b: int(lens_k[b])  # noqa: E731  (q_len rows see <= Lk keys; decode sees Lk)
@@ -350,9 +368,24 @@ def cpu_baseline(batch: W.Batch, bytes_: dict, budget_s: float = 20.0) -> dict:
     work_all = sum(vis(b) for b in rows_all[:, 0])
     frac = work_sel / max(work_all, 1)
     value = bytes_["total"] * frac / t / 1e9
-    return {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+    return {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{len(sel)} of {len(rows_all)} output rows ({100 * frac:.1f}% of the row x key work), "
                       f"median of 3, scaled to the whole call"}
+
+
+def cpu_baseline_steps(name: str, batch: W.Batch, budget_s: float, steps=(0, 49, 99)) -> dict:
+    """Continuous batching: the oracle at several length draws of the same
+    K/V buffer, each a bounded sample; reports the mean GB/s per step."""
+    draws = W.lengths(name, seed=0)
+    per = []
+    for s in steps:
+        lq, lk = draws[s]
+        b = W.Batch(batch.shape, batch.q[: int(lq.sum())], batch.k, batch.v, W.cu_from_lengths(lq),
+                    W.cu_from_lengths(lk), lq, lk)
+        per.append(cpu_baseline(b, algorithmic_bytes(b), budget_s / len(steps), seed=1 + s))
+    return {"value": statistics.mean(p["value"] for p in per), "unit": "GB/s", "cores": per[0]["cores"],
+            "kind": "oracle", "steps": list(steps), "per_step": [p["value"] for p in per],
+            "sample": "length draws " + ", ".join(str(s) for s in steps) + ": " + "; ".join(p["sample"] for p in per)}
 
 
 # ------------------------------------------------------------------ our arm
@@ -380,130 +413,233 @@ def step_cu_k(name: str, batch: W.Batch):
     return np.stack(cus), byts
 
 
+def max_over_ranks_vec(xs, pg) -> list:
+    """Element-wise max over ranks of a list of floats (one collective)."""
+    if pg is None:
+        return list(xs)
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(list(xs), dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+KERNELS = {1: "split_simt_kernel", 2: "split_mma_kernel", 3: "split_tc_kernel"}
+MIN_TIMED_S = 0.25          # timed passes repeat until about this much device time
+MAX_PASSES = 400
+
+
+class Workload:
+    """One workload on one GPU: inputs resident in HBM, a plan, and CUDA
+    graphs of its calls, ready to be timed."""
+
+    def __init__(self, name, args, dev, page_size=0):
+        from varlen_gqa_split_b200 import Plan
+        self.name, self.dev, self.page_size = name, dev, page_size
+        batch = make_inputs(name, dev)
+        sh = batch.shape
+        self.batch, self.sh = batch, sh
+        self.bytes = algorithmic_bytes(batch)
+        q, k, v = batch.q, batch.k, batch.v
+        self.paged = None
+        if page_size:
+            # the same keys in a paged cache: shuffled pages of page_size tokens,
+            # one block-table row per sequence (only step 0's lengths are placed,
+            # so one draw of lengths)
+            if name == "continuous":
+                raise SystemExit("--page-size: the continuous workload changes its lengths every step")
+            self.paged = W.paginate(k, v, batch.cu_k, sh.B, page_size, sh.s_max, seed=0, fill=0.0)
+            k, v = self.paged.k_cache, self.paged.v_cache
+        self.q, self.k, self.v = q, k, v
+        self.cu_q = torch.from_numpy(batch.cu_q).to(dev)
+        self.cu_k = torch.from_numpy(batch.cu_k).to(dev)
+        self.out = torch.empty_like(q)
+        self.lse = torch.empty(q.shape[0], sh.Hq, dtype=torch.float32, device=dev)
+        self.plan = Plan(sh.B, sh.s_max, sh.Hq, sh.Hkv, sh.D, sh.max_q, nsplit=args.nsplit, variant=args.variant,
+                         stages=args.stages, combine=args.combine, ctas=args.ctas,
+                         deterministic=int(args.deterministic))
+        self.info = self.plan.info
+        self.launches_per_call = 2 if self.info["combine"] == 1 else 1     # split (+ combine kernel)
+        self.kernel = KERNELS[self.info["variant"]]
+        self.stream = torch.cuda.Stream(dev)
+        # A call whose inputs exceed L2 is timed in a pipeline: R copies of the
+        # inputs (together several times L2), one per layer of a model, and one
+        # CUDA graph holding R calls, one per copy -- the attention calls of a
+        # decode step over the layers' own caches.  K calls = K/R replays (plus
+        # a shorter graph for a remainder) between one pair of events.  A
+        # smaller call is timed alone: L2 flushed before each call, events
+        # captured inside the graph around the call.  The isolated per-call
+        # latency (flush, then one call) is reported for every workload.
+        cu_steps_h, self.step_bytes = step_cu_k(name, batch)
+        self.n_var = len(self.step_bytes)
+        self.pipelined = min(self.step_bytes) >= L2_BYTES
+        n_copies = max(2, min(8, -(-4 * L2_BYTES // min(self.step_bytes)))) if self.pipelined else 1
+        self.n_copies = n_copies
+        self.copies = [(q, k, v, self.out, self.lse)]
+        for _ in range(n_copies - 1):
+            self.copies.append((q.clone(), k.clone(), v.clone(), torch.empty_like(self.out),
+                                torch.empty_like(self.lse)))
+        # one cu_seqlens_k row per copy; with several length draws, the rows of
+        # the next n_copies draws are written in place before each replay
+        cu_ext = np.concatenate([cu_steps_h, cu_steps_h[:n_copies]]) if self.n_var > 1 else cu_steps_h
+        self.cu_steps = torch.from_numpy(cu_ext).to(dev)
+        self.cu_rows = self.cu_steps[:1].repeat(n_copies, 1).contiguous()
+        self.in0 = torch.cuda.Event(enable_timing=True, external=True)
+        self.in1 = torch.cuda.Event(enable_timing=True, external=True)
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.graphs = {}
+        with torch.cuda.stream(self.stream):
+            self.call(q, k, v, self.cu_q, self.cu_rows[0], self.out, self.lse)
+            self.stream.synchronize()
+            self.g_iso = self._capture(1, events=True)
+            self.g_all = self._capture(n_copies) if self.pipelined else None
+
+    def call(self, qq, kk, vv, cq, ck, oo, ll):
+        if self.paged is None:
+            return self.plan.run(qq, kk, vv, cq, ck, oo, ll)
+        return self.plan.run_paged(qq, kk, vv, self.paged.block_table, cq, ck, oo, ll)
+
+    def _capture(self, n_calls, events=False):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream, capture_error_mode="global"):
+            if events:
+                self.in0.record(self.stream)
+            for r in range(n_calls):
+                qq, kk, vv, oo, ll = self.copies[r]
+                self.call(qq, kk, vv, self.cu_q, self.cu_rows[r], oo, ll)
+            if events:
+                self.in1.record(self.stream)
+        return g
+
+    def rem_graph(self, steps):
+        rem = steps % self.n_copies
+        if not (self.pipelined and rem):
+            return None
+        if rem not in self.graphs:
+            with torch.cuda.stream(self.stream):
+                self.graphs[rem] = self._capture(rem)
+        return self.graphs[rem]
+
+    def isolated_step(self):
+        self.flush.zero_()
+        self.g_iso.replay()
+        self.stream.synchronize()
+        return self.in0.elapsed_time(self.in1)
+
+    def set_draws(self, j):
+        if self.n_var > 1:
+            s0 = (j * self.n_copies) % self.n_var
+            self.cu_rows.copy_(self.cu_steps[s0:s0 + self.n_copies], non_blocking=True)
+
+    def timed_pass(self, steps, pg):
+        """One timed pass of exactly `steps` calls (barrier + synchronise on
+        both sides); returns this rank's milliseconds."""
+        g_rem = self.rem_graph(steps)
+        o0 = torch.cuda.Event(enable_timing=True)
+        o1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            self.stream.synchronize()
+            barrier(pg)
+            torch.cuda.synchronize(self.dev)
+            if self.pipelined:
+                o0.record(self.stream)
+                for j in range(steps // self.n_copies):
+                    self.set_draws(j)
+                    self.g_all.replay()
+                if g_rem is not None:
+                    self.set_draws(steps // self.n_copies)
+                    g_rem.replay()
+                o1.record(self.stream)
+                self.stream.synchronize()
+                ms = o0.elapsed_time(o1)
+            else:
+                ms = sum(self.isolated_step() for _ in range(steps))
+            torch.cuda.synchronize(self.dev)
+            barrier(pg)
+        return ms
+
+    def bytes_of(self, steps):
+        if self.pipelined:
+            return sum(self.step_bytes[i % self.n_var] for i in range(steps))
+        return self.bytes["total"] * steps
+
+    def measure(self, steps, warmup, pg, n_iso=200, min_timed_s=MIN_TIMED_S):
+        """Warm-up, isolated calls, then repeated timed passes of `steps` calls
+        (the same number of passes on every rank), clocks sampled throughout.
+        Returns the per-pass milliseconds (max over ranks), the isolated-call
+        milliseconds and the clock summary."""
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                self.isolated_step()
+            iso_ms = [self.isolated_step() for _ in range(min(steps, n_iso))]
+            if self.pipelined:
+                for j in range(warmup):
+                    self.set_draws(j)
+                    self.g_all.replay()
+            self.stream.synchronize()
+        first = self.timed_pass(steps, pg)
+        n_pass = int(min(MAX_PASSES, max(5, math.ceil(min_timed_s * 1e3 / max(first, 1e-3)))))
+        n_pass = int(max_over_ranks(float(n_pass), pg))
+        local = []
+        with ClockSampler(self.dev.index if self.dev.index is not None else 0) as clocks:
+            for _ in range(n_pass):
+                local.append(self.timed_pass(steps, pg))
+        passes = max_over_ranks_vec(local, pg)
+        assert self.plan.check_error() == 0, "device error flag set during the benchmark"
+        return passes, iso_ms, clocks.summary()
+
+    def summary(self, steps, passes, iso_ms, clocks, world) -> dict:
+        """us per call, GB/s and roofline fraction from the median pass."""
+        med = statistics.median(passes)
+        q10, q90 = np.percentile(passes, [10, 90])
+        timed_bytes = self.bytes_of(steps)
+        achieved = timed_bytes / (med * 1e-3) / 1e9
+        peak, peak_src = measured_peak()
+        traffic_key = self.name + (f"_paged{self.page_size}" if self.paged is not None else "")
+        traffic, traffic_note = recorded_traffic(traffic_key, self.kernel)
+        us = 1e3 * med / steps
+        d = {"us_per_call": us, "value_gbs": achieved * world, "frac": achieved / peak,
+             "kernel": self.kernel, "calls_per_pass": steps, "passes": len(passes),
+             "us_per_call_p10_p90": [1e3 * q10 / steps, 1e3 * q90 / steps],
+             "us_per_call_min_max": [1e3 * min(passes) / steps, 1e3 * max(passes) / steps],
+             "bytes_per_call": timed_bytes / steps, "length_draws_cycled": self.n_var,
+             "traffic": traffic, "clocks": clocks,
+             "isolated_call_us": {"median": 1e3 * statistics.median(iso_ms), "min": 1e3 * min(iso_ms),
+                                  "max": 1e3 * max(iso_ms), "calls": len(iso_ms),
+                                  "value_gbs": self.bytes["total"] / (statistics.median(iso_ms) * 1e-3) / 1e9}}
+        if clocks.get("sm_mhz"):
+            d["kcycles_per_call"] = us * clocks["sm_mhz"] / 1e3
+        if traffic is None:
+            d["traffic_note"] = traffic_note
+        if self.name == "prefill":
+            flops = attention_flops(self.batch)
+            tpeak, _ = measured_tensor_peak()
+            d["tflops"] = flops / (us * 1e-6) / 1e12
+            d["tensor_frac"] = d["tflops"] / tpeak
+        return d, achieved, peak, peak_src, traffic, traffic_note
+
+    def close(self):
+        self.g_iso = self.g_all = None
+        self.graphs.clear()
+        self.plan.close()
+
+
+# the workloads the method's ≥70% target names, and the short-query one it
+# also asks to report; measured beside the headline workload in one run
+EXTRA_WORKLOADS = ("ragged", "continuous", "shortq", "tiny")
+
+
 def run_ours(args, rank, world, local, pg) -> dict | None:
-    from varlen_gqa_split_b200 import Plan, build
+    from varlen_gqa_split_b200 import build
     build.build()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    batch = make_inputs(args.workload, dev)
-    sh = batch.shape
-    bytes_ = algorithmic_bytes(batch)
-    q, k, v = batch.q, batch.k, batch.v
-    paged = None
-    if args.page_size:
-        # the same keys in a paged cache: shuffled pages of page_size tokens,
-        # one block-table row per sequence (only step 0's lengths are placed,
-        # so one draw of lengths)
-        if args.workload == "continuous":
-            raise SystemExit("--page-size: the continuous workload changes its lengths every step")
-        paged = W.paginate(k, v, batch.cu_k, sh.B, args.page_size, sh.s_max, seed=0, fill=0.0)
-        k, v = paged.k_cache, paged.v_cache
-    cu_q = torch.from_numpy(batch.cu_q).to(dev)
-    cu_k = torch.from_numpy(batch.cu_k).to(dev)
-    out = torch.empty_like(q)
-    lse = torch.empty(q.shape[0], sh.Hq, dtype=torch.float32, device=dev)
-    plan = Plan(sh.B, sh.s_max, sh.Hq, sh.Hkv, sh.D, sh.max_q, nsplit=args.nsplit, variant=args.variant,
-                stages=args.stages, combine=args.combine, ctas=args.ctas,
-                deterministic=int(args.deterministic))
-    info = plan.info
-    launches_per_call = 2 if info["combine"] == 1 else 1     # split (+ combine kernel)
-
-    stream = torch.cuda.Stream(dev)
-    # Timing.  A call whose inputs exceed L2 is timed in a pipeline: R copies
-    # of the inputs (together several times L2), one per layer of a model, and
-    # one CUDA graph holding R calls, one per copy -- the attention calls of a
-    # decode step over the layers' own caches.  K calls = K/R replays (plus a
-    # shorter graph for a remainder) between one pair of events.  A smaller
-    # call is timed alone: L2 flushed before each call, events captured inside
-    # the graph around the call.  The isolated per-call latency (flush, then
-    # one call) is reported for every workload.
-    cu_steps_h, step_bytes = step_cu_k(args.workload, batch)
-    n_var = len(step_bytes)
-    pipelined = min(step_bytes) >= L2_BYTES
-    n_copies = max(2, min(8, -(-4 * L2_BYTES // min(step_bytes)))) if pipelined else 1
-    copies = [(q, k, v, out, lse)]
-    for _ in range(n_copies - 1):
-        copies.append((q.clone(), k.clone(), v.clone(), torch.empty_like(out), torch.empty_like(lse)))
-    # one cu_seqlens_k row per copy; with several length draws, the rows of
-    # the next n_copies draws are written in place before each replay
-    cu_ext = np.concatenate([cu_steps_h, cu_steps_h[:n_copies]]) if n_var > 1 else cu_steps_h
-    cu_steps = torch.from_numpy(cu_ext).to(dev)
-    cu_rows = cu_steps[:1].repeat(n_copies, 1).contiguous()
-    in0 = torch.cuda.Event(enable_timing=True, external=True)
-    in1 = torch.cuda.Event(enable_timing=True, external=True)
-
-    def call(qq, kk, vv, cq, ck, oo, ll):
-        if paged is None:
-            return plan.run(qq, kk, vv, cq, ck, oo, ll)
-        return plan.run_paged(qq, kk, vv, paged.block_table, cq, ck, oo, ll)
-
-    def capture(n_calls, events=False):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="global"):
-            if events:
-                in0.record(stream)
-            for r in range(n_calls):
-                qq, kk, vv, oo, ll = copies[r]
-                call(qq, kk, vv, cu_q, cu_rows[r], oo, ll)
-            if events:
-                in1.record(stream)
-        return g
-
-    with torch.cuda.stream(stream):
-        call(q, k, v, cu_q, cu_rows[0], out, lse)
-        stream.synchronize()
-        g_iso = capture(1, events=True)
-        g_all = capture(n_copies) if pipelined else None
-        rem = args.steps % n_copies
-        g_rem = capture(rem) if pipelined and rem else None
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    o0 = torch.cuda.Event(enable_timing=True)
-    o1 = torch.cuda.Event(enable_timing=True)
-
-    def isolated_step():
-        flush.zero_()
-        g_iso.replay()
-        stream.synchronize()
-        return in0.elapsed_time(in1)
-
-    def set_draws(j):
-        if n_var > 1:
-            s0 = (j * n_copies) % n_var
-            cu_rows.copy_(cu_steps[s0:s0 + n_copies], non_blocking=True)
-
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            isolated_step()
-        iso_ms = [isolated_step() for _ in range(min(args.steps, 200))]
-        if pipelined:
-            for j in range(args.warmup):
-                set_draws(j)
-                g_all.replay()
-        stream.synchronize()
-        barrier(pg)
-        torch.cuda.synchronize(dev)
-        with ClockSampler(local) as clocks:
-            if pipelined:
-                o0.record(stream)
-                for j in range(args.steps // n_copies):
-                    set_draws(j)
-                    g_all.replay()
-                if g_rem is not None:
-                    set_draws(args.steps // n_copies)
-                    g_rem.replay()
-                o1.record(stream)
-                stream.synchronize()
-                total_local_ms = o0.elapsed_time(o1)
-            else:
-                total_local_ms = sum(isolated_step() for _ in range(args.steps))
-        torch.cuda.synchronize(dev)
-        barrier(pg)
-    total_ms = max_over_ranks(total_local_ms, pg)
-    ms_per_step = total_ms / args.steps
-    timed_bytes = (sum(step_bytes[i % n_var] for i in range(args.steps)) if pipelined
-                   else bytes_["total"] * args.steps)
-    value = timed_bytes * world / (total_ms * 1e-3) / 1e9
-    assert plan.check_error() == 0, "device error flag set during the benchmark"
+    wl = Workload(args.workload, args, dev, args.page_size)
+    sh, info, batch, bytes_ = wl.sh, wl.info, wl.batch, wl.bytes
+    passes, iso_ms, clocks = wl.measure(args.steps, args.warmup, pg)
+    ws, achieved, peak, peak_src, traffic, traffic_note = wl.summary(args.steps, passes, iso_ms, clocks, world)
+    ms_per_step = statistics.median(passes) / args.steps
+    value = ws["value_gbs"]
+    timed_bytes = wl.bytes_of(args.steps)
 
     # roofline of the split kernel.  One call is one split-kernel launch,
     # followed on the tensor-core path by the LSE combine kernel, launched as a
@@ -512,24 +648,19 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     # achieved figure charges the combine tail to the split kernel: a lower
     # bound on the split kernel's own rate.  Its share of device time is in the
     # committed ncu launch list.
-    peak, peak_src = measured_peak()
-    kernel = {1: "split_simt_kernel", 2: "split_mma_kernel", 3: "split_tc_kernel"}[info["variant"]]
-    achieved = timed_bytes / (total_ms * 1e-3) / 1e9
-    traffic_key = args.workload + (f"_paged{args.page_size}" if paged is not None else "")
-    traffic, traffic_note = recorded_traffic(traffic_key, kernel)
-    roofline = {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",
+    roofline = {"bound": "hbm", "kernel": wl.kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": timed_bytes / args.steps,
                 "timed": ("one call: split kernel + LSE combine kernel (programmatic dependent launch)"
-                          if launches_per_call == 2 else "one call: the split kernel alone")}
+                          if wl.launches_per_call == 2 else "one call: the split kernel alone")}
     if traffic is None:
         roofline["traffic_note"] = traffic_note
     if args.workload == "prefill":
         # queries of up to 2048 tokens: the contraction, not HBM, bounds it
         flops = attention_flops(batch)
         tpeak, tsrc = measured_tensor_peak()
-        tach = flops / (total_ms / args.steps * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "kernel": kernel, "achieved": tach, "peak": tpeak, "unit": "TFLOP/s",
+        tach = flops / (ms_per_step * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": wl.kernel, "achieved": tach, "peak": tpeak, "unit": "TFLOP/s",
                     "frac": tach / tpeak, "traffic": traffic, "peak_source": tsrc,
                     "algorithmic_flops_per_launch": flops, "hbm_gbs": achieved,
                     "timed": roofline["timed"]}
@@ -537,59 +668,38 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        n_e2e = max(3, min(args.steps, 20))
-        # only the tokens this step's lengths cover cross the bus
-        tkv = batch.kv_tokens if paged is None else k.shape[0]
-        hq = batch.q.cpu().pin_memory()
-        hk = k[:tkv].cpu().pin_memory()
-        hv = v[:tkv].cpu().pin_memory()
-        hcq = torch.from_numpy(batch.cu_q).pin_memory()
-        hck = torch.from_numpy(batch.cu_k).pin_memory()
-        ho = torch.empty_like(hq).pin_memory()
-        hl = torch.empty(hq.shape[0], sh.Hq, dtype=torch.float32).pin_memory()
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        if paged is not None:
-            # the halves of one buffer stay views of one buffer
-            dk, dv = torch.empty_like(k.contiguous()), torch.empty_like(v.contiguous())
-            hbt = paged.block_table.cpu().pin_memory()
-            dbt = torch.empty_like(paged.block_table)
-        dcq, dck = torch.empty_like(cu_q), torch.empty_like(cu_k)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
-        if paged is not None:
-            h2d += hbt.numel() * hbt.element_size()
-        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
-        with torch.cuda.stream(stream):
-            def e2e_step():
-                dq.copy_(hq, non_blocking=True)
-                dk[:tkv].copy_(hk, non_blocking=True)
-                dv[:tkv].copy_(hv, non_blocking=True)
-                dcq.copy_(hcq, non_blocking=True)
-                dck.copy_(hck, non_blocking=True)
-                if paged is None:
-                    o, l_ = plan.run(dq, dk, dv, dcq, dck, out, lse)
-                else:
-                    dbt.copy_(hbt, non_blocking=True)
-                    o, l_ = plan.run_paged(dq, dk, dv, dbt, dcq, dck, out, lse)
-                ho.copy_(o, non_blocking=True)
-                hl.copy_(l_, non_blocking=True)
-            for _ in range(2):
-                e2e_step()
-            stream.synchronize()
-            barrier(pg)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(n_e2e):
-                e2e_step()
-            e1.record(stream)
-            stream.synchronize()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg)
-        e2e = {"value": bytes_["total"] * n_e2e * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "us_per_call": 1e3 * e2e_ms / n_e2e}
+        e2e = measure_e2e(wl, args, pg, world)
+
+    # the other workloads of the method, in the same process (one GPU)
+    extras = {}
+    if not args.only and world == 1 and args.page_size == 0:
+        for name in EXTRA_WORKLOADS:
+            if name == args.workload:
+                continue
+            other = Workload(name, args, dev)
+            # continuous batching: one pass walks all 100 length draws
+            st = other.n_var if other.n_var > 1 else args.steps
+            p_, iso_, clk_ = other.measure(st, args.warmup, pg, n_iso=50)
+            extras[name], *_ = other.summary(st, p_, iso_, clk_, world)
+            extras[name]["workload"] = DESCRIPTIONS[name]
+            extras[name]["plan"] = {kk: other.info[kk] for kk in ("variant", "ctas", "stages", "combine")}
+            if name == "tiny":
+                extras[name]["note"] = "latency-bound (37 KB per call): timed alone after an L2 flush"
+            if rank == 0 and not args.no_cpu_baseline:
+                if name == "continuous":
+                    extras[name]["cpu_baseline"] = cpu_baseline_steps(name, other.batch, 12.0)
+                elif name != "tiny":
+                    extras[name]["cpu_baseline"] = cpu_baseline(other.batch, other.bytes, 8.0)
+            other.close()
+            del other
+            torch.cuda.empty_cache()
 
     res = None
     if rank == 0:
-        cpu = None if (args.no_cpu_baseline or world > 1) else cpu_baseline(batch, bytes_)
+        cpu = None
+        if not (args.no_cpu_baseline or world > 1):
+            cpu = cpu_baseline(batch, bytes_)
+            cpu["single_thread"] = cpu_baseline(batch, bytes_, budget_s=8.0, threads=1)
         res = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_call": 1e3 * ms_per_step,
@@ -598,37 +708,98 @@ def run_ours(args, rank, world, local, pg) -> dict | None:
             "config": {"workload": DESCRIPTIONS[args.workload], "B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv,
                        "D": sh.D, "max_q": sh.max_q, "s_max": sh.s_max,
                        "kv_tokens": int(batch.lens_k.sum()), "q_tokens": int(batch.lens_q.sum()),
-                       "kv_layout": ("packed THD" if paged is None else
-                                     f"paged: {k.shape[0]} pages of {args.page_size} tokens in shuffled "
+                       "kv_layout": ("packed THD" if wl.paged is None else
+                                     f"paged: {wl.k.shape[0]} pages of {args.page_size} tokens in shuffled "
                                      f"order, one block-table row per sequence"),
                        "bytes_per_call": timed_bytes / args.steps, "lse_bytes_per_call": bytes_["lse"],
-                       "length_draws_cycled": n_var,
-                       "l2": (f"inputs larger than L2: {n_copies} copies of the inputs ({n_copies} x "
-                              f"{bytes_['total'] / 1e6:.0f} MB) used in turn" if pipelined else
+                       "length_draws_cycled": wl.n_var,
+                       "l2": (f"inputs larger than L2: {wl.n_copies} copies of the inputs ({wl.n_copies} x "
+                              f"{bytes_['total'] / 1e6:.0f} MB) used in turn" if wl.pipelined else
                               "flushed before every timed call (512 MB write, outside the timed events)"),
-                       "timing": (f"CUDA events around K attn_run calls, captured {n_copies} per CUDA graph "
+                       "timing": (f"CUDA events around K attn_run calls, captured {wl.n_copies} per CUDA graph "
                                   f"(one per input copy, like the layers of a decode step) and replayed back "
                                   f"to back" +
                                   ("; before each replay one device-to-device copy writes the next draws' "
-                                   "cu_seqlens_k in place (timed)" if n_var > 1 else "") if pipelined else
+                                   "cu_seqlens_k in place (timed)" if wl.n_var > 1 else "") if wl.pipelined else
                                   "CUDA events captured inside the graph around the attn_run call, one replay "
-                                  "per step after an L2 flush, summed"),
+                                  "per step after an L2 flush, summed") +
+                                 f"; {len(passes)} timed passes of K = {args.steps} calls, each bracketed by a "
+                                 f"barrier and synchronisation, value from the median pass",
                        "parallelism": f"replicas x{world} (independent sequences)",
                        "plan": {kk: info[kk] for kk in ("variant", "nsplit", "chunk", "ctas", "stages", "grid_x",
                                                          "grid_y", "grid_z", "combine", "smem_bytes")}},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches_per_call * args.steps,
-            "clocks": clocks.summary(),
-            "isolated_call_us": {"median": 1e3 * statistics.median(iso_ms), "min": 1e3 * min(iso_ms),
-                                 "max": 1e3 * max(iso_ms),
-                                 "value_gbs": bytes_["total"] / (statistics.median(iso_ms) * 1e-3) / 1e9,
-                                 "how": "L2 flushed, then one call; CUDA events inside the captured graph"},
+            "gpu_launches": wl.launches_per_call * args.steps,
+            "clocks": clocks,
+            "passes": {k_: ws[k_] for k_ in ("passes", "us_per_call_p10_p90", "us_per_call_min_max")},
+            "isolated_call_us": ws["isolated_call_us"],
         }
-    del g_iso, g_all, g_rem
-    plan.close()
+        if "kcycles_per_call" in ws:
+            res["kcycles_per_call"] = ws["kcycles_per_call"]
+        if extras:
+            res["workloads"] = extras
+    wl.close()
     return res
+
+
+def measure_e2e(wl: Workload, args, pg, world) -> dict:
+    """The same call end to end through the public API: pinned host buffers,
+    the host-to-device copies of the step's inputs and the device-to-host
+    copies of its outputs inside the timed region."""
+    batch, sh, plan, paged = wl.batch, wl.sh, wl.plan, wl.paged
+    k, v, q = wl.k, wl.v, wl.q
+    n_e2e = max(3, min(args.steps, 20))
+    # only the tokens this step's lengths cover cross the bus
+    tkv = batch.kv_tokens if paged is None else k.shape[0]
+    hq = batch.q.cpu().pin_memory()
+    hk = k[:tkv].cpu().pin_memory()
+    hv = v[:tkv].cpu().pin_memory()
+    hcq = torch.from_numpy(batch.cu_q).pin_memory()
+    hck = torch.from_numpy(batch.cu_k).pin_memory()
+    ho = torch.empty_like(hq).pin_memory()
+    hl = torch.empty(hq.shape[0], sh.Hq, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if paged is not None:
+        # the halves of one buffer stay views of one buffer
+        dk, dv = torch.empty_like(k.contiguous()), torch.empty_like(v.contiguous())
+        hbt = paged.block_table.cpu().pin_memory()
+        dbt = torch.empty_like(paged.block_table)
+    dcq, dck = torch.empty_like(wl.cu_q), torch.empty_like(wl.cu_k)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
+    if paged is not None:
+        h2d += hbt.numel() * hbt.element_size()
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    stream = wl.stream
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk[:tkv].copy_(hk, non_blocking=True)
+            dv[:tkv].copy_(hv, non_blocking=True)
+            dcq.copy_(hcq, non_blocking=True)
+            dck.copy_(hck, non_blocking=True)
+            if paged is None:
+                o, l_ = plan.run(dq, dk, dv, dcq, dck, wl.out, wl.lse)
+            else:
+                dbt.copy_(hbt, non_blocking=True)
+                o, l_ = plan.run_paged(dq, dk, dv, dbt, dcq, dck, wl.out, wl.lse)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(l_, non_blocking=True)
+        for _ in range(2):
+            e2e_step()
+        stream.synchronize()
+        barrier(pg)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg)
+    return {"value": wl.bytes["total"] * n_e2e * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+            "us_per_call": 1e3 * e2e_ms / n_e2e}
 
 
 def main():
@@ -648,6 +819,8 @@ def main():
     ap.add_argument("--page-size", type=int, default=0,
                     help="read K/V from a paged cache with pages of this many tokens (0: packed)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", action="store_true",
+                    help="time the selected workload alone (no other workloads in the same run)")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -99,6 +99,17 @@ typedef struct {
                           0: the plan's choice: run-time balancing on the
                           warp-MMA path, static shares on the tcgen05 path
                           (the CUDA-core path is always repeatable)           */
+    int wait_limit_us; /* upper bound of one bounded device wait (a pipeline
+                          stage, a merge waiting for a unit's parts), in
+                          microseconds; 0 keeps the default of 2 s.  A wait
+                          that runs out sets ATTN_DEV_ERR_TIMEOUT and its block
+                          returns without writing the rows it was to write  */
+    int test_stall;    /* test hook, tensor-core paths only: 1 makes the merge
+                          of every cut unit wait for one part that is never
+                          written, so those waits run out (after
+                          wait_limit_us) on the plan's first call, leaving the
+                          cut units' rows unwritten; attn_check_error() clears
+                          it.  0 in every other use                         */
 } attn_overrides;
 
 /* What the planner chose (attn_plan_info). */
@@ -289,7 +300,9 @@ int attn_merge_lse(int n_parts, const void *outs, const float *lses, int64_t T_q
  * attn_check_error -- synchronise `stream`, then read and clear the plan's
  * sticky device error bits (ATTN_DEV_ERR_*) into *flags.  When a bit was set
  * it also resets the plan's merge tickets, so the plan stays usable after a
- * call that stopped early.  The only entry point that waits for the GPU; do
+ * call that stopped early (for instance one whose bounded waits ran out:
+ * ATTN_DEV_ERR_TIMEOUT; see attn_overrides.wait_limit_us).  It also clears
+ * the attn_overrides.test_stall hook.  The only entry point that waits for the GPU; do
  * not call it inside stream capture.
  */
 int attn_check_error(attn_plan_t plan, void *stream, uint32_t *flags);
@@ -325,6 +338,11 @@ const char *attn_strerror(int code);
  *
  * The first call on each device looks up the array's device address and sets
  * a kernel attribute; make that first call before any stream capture begins.
+ * With CUDA's lazy module loading (the default since CUDA 12.2) the array's
+ * device memory is committed at that first call, not when the library is
+ * loaded: a caller whose pool allocator reserves the device's memory should
+ * make the first call on each device before the pool takes its reservation,
+ * or the first call can fail with ATTN_E_CUDA.
  * All calls on a device share the array and leave their contents in it; each
  * call clears the parts that must start at zero on its own stream.  Calls
  * that overlap on the GPU race on the array: order them (one stream, or

@@ -104,6 +104,13 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's later OpenMP regions (for a single-thread
+    baseline).  Sets the OpenMP runtime the oracle library is linked with."""
+    _load()
+    ctypes.CDLL("libgomp.so.1").omp_set_num_threads(ctypes.c_int(int(n)))
+
+
 def attention(q, k, v, cu_q, cu_k, *, B, Hq, Hkv, D, scale=None, causal=True,
               out=None, lse=None):
     """Whole-batch attention.

@@ -2,6 +2,8 @@
 compare with the fp64 oracle on the same bytes."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -13,6 +15,65 @@ from varlen_gqa_split_b200 import Plan
 # absolute, against the fp64 definition
 ATOL_OUT = 2e-2
 ATOL_LSE = 1e-3
+# and per output row (one query token and head): ||out - ref||_2 / ||ref||_2.
+# At long contexts the output itself is small (rms ~0.01 over 32768 keys), so
+# the absolute bound alone would pass a row that is wrong by 100%; this bound
+# does not.  Rounding the output to bf16 alone costs ~1e-3.
+RTOL_ROW = 1e-2
+
+# measured errors of every comparison in this session, printed at the end of
+# the run (conftest.pytest_terminal_summary): label -> [rows, max |out err|,
+# max row relative err, max |lse err|]
+ERRORS: dict = {}
+
+
+def _label(label):
+    if label:
+        return label
+    cur = os.environ.get("PYTEST_CURRENT_TEST", "?")
+    return cur.split(" ")[0]
+
+
+def record(label, n_rows, err_o, rel_o, err_l):
+    e = ERRORS.setdefault(_label(label), [0, 0.0, 0.0, 0.0])
+    e[0] += int(n_rows)
+    e[1] = max(e[1], float(err_o))
+    e[2] = max(e[2], float(rel_o))
+    e[3] = max(e[3], float(err_l))
+
+
+def row_rel_err(o, ro):
+    """max over rows (last axis = D) of ||o - ro|| / ||ro||, for rows whose
+    reference is not exactly zero (no visible key)."""
+    o = np.asarray(o, dtype=np.float64).reshape(-1, ro.shape[-1])
+    ro = np.asarray(ro, dtype=np.float64).reshape(-1, ro.shape[-1])
+    nref = np.linalg.norm(ro, axis=1)
+    live = nref > 0
+    if not live.any():
+        return 0.0
+    return float((np.linalg.norm(o[live] - ro[live], axis=1) / nref[live]).max())
+
+
+def check_values(o, l, ro, rl, label=None, atol_out=ATOL_OUT, atol_lse=ATOL_LSE, rtol_row=RTOL_ROW):
+    """out rows o [..., D] and lse l [...] against the oracle's ro, rl: max-abs
+    on both, per-row relative error on out, -inf lse (and a zero row there)
+    matched exactly.  Records and returns (max |out err|, max row rel err,
+    max |lse err|)."""
+    o = np.asarray(o, dtype=np.float64)
+    l = np.asarray(l, dtype=np.float64)
+    assert np.all(np.isfinite(o)), "non-finite output in a checked row"
+    err_o = float(np.abs(o - ro).max()) if o.size else 0.0
+    rel_o = row_rel_err(o, ro) if o.size else 0.0
+    ninf_ref = np.isneginf(rl)
+    assert np.array_equal(np.isneginf(l), ninf_ref), "-inf lse pattern differs from the oracle"
+    assert np.all(o[ninf_ref] == 0.0), "rows with no visible key must be exactly 0"
+    fin = ~ninf_ref
+    err_l = float(np.abs(l[fin] - rl[fin]).max()) if fin.any() else 0.0
+    record(label, l.size, err_o, rel_o, err_l)
+    assert err_o <= atol_out, f"max |out - oracle| = {err_o}"
+    assert rel_o <= rtol_row, f"max row ||out - oracle|| / ||oracle|| = {rel_o}"
+    assert err_l <= atol_lse, f"max |lse - oracle| = {err_l}"
+    return err_o, rel_o, err_l
 
 BF16_NAN_BITS = 0x7FC0
 
@@ -68,7 +129,8 @@ def covered_rows(batch: W.Batch) -> np.ndarray:
     return m
 
 
-def compare_full(out_gpu, lse_gpu, out_ref, lse_ref, covered, atol_out=ATOL_OUT, atol_lse=ATOL_LSE):
+def compare_full(out_gpu, lse_gpu, out_ref, lse_ref, covered, atol_out=ATOL_OUT, atol_lse=ATOL_LSE,
+                 label=None):
     """Element-wise check of every covered row; rows not covered must keep
     the NaN sentinel bit pattern.  Returns (max |out err|, max |lse err|)."""
     o = out_gpu.float().numpy().astype(np.float64)
@@ -76,15 +138,7 @@ def compare_full(out_gpu, lse_gpu, out_ref, lse_ref, covered, atol_out=ATOL_OUT,
     T = covered.shape[0]
     oc, lc = o[:T][covered], l[:T][covered]
     ro, rl = out_ref[:T][covered], lse_ref[:T][covered]
-    assert np.all(np.isfinite(oc)), "non-finite output in a covered row"
-    err_o = np.abs(oc - ro).max() if oc.size else 0.0
-    assert err_o <= atol_out, f"max |out - oracle| = {err_o}"
-    ninf_ref = np.isneginf(rl)
-    assert np.array_equal(np.isneginf(lc), ninf_ref), "-inf lse pattern differs from the oracle"
-    assert np.all(oc[ninf_ref] == 0.0), "rows with no visible key must be exactly 0"
-    fin = ~ninf_ref
-    err_l = np.abs(lc[fin] - rl[fin]).max() if fin.any() else 0.0
-    assert err_l <= atol_lse, f"max |lse - oracle| = {err_l}"
+    err_o, _, err_l = check_values(oc, lc, ro, rl, label, atol_out, atol_lse)
     # untouched rows: bitwise sentinel
     raw = out_gpu.view(torch.int16).numpy()
     untouched = np.ones(raw.shape[0], dtype=bool)
@@ -110,7 +164,7 @@ def sample_rows(batch: W.Batch, n, rng):
     return np.array(sorted(rows), dtype=np.int64).reshape(-1, 3)
 
 
-def compare_rows(out_gpu, lse_gpu, batch: W.Batch, rows, atol_out=ATOL_OUT, atol_lse=ATOL_LSE):
+def compare_rows(out_gpu, lse_gpu, batch: W.Batch, rows, atol_out=ATOL_OUT, atol_lse=ATOL_LSE, label=None):
     sh = batch.shape
     ro, rl = oracle.attention_rows(W.bits(batch.q), W.bits(batch.k), W.bits(batch.v), batch.cu_q,
                                    batch.cu_k, rows, B=sh.B, Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D,
@@ -118,12 +172,7 @@ def compare_rows(out_gpu, lse_gpu, batch: W.Batch, rows, atol_out=ATOL_OUT, atol
     tok = batch.cu_q[rows[:, 0]] + rows[:, 1]
     o = out_gpu[tok, rows[:, 2]].float().numpy().astype(np.float64)
     l = lse_gpu[tok, rows[:, 2]].numpy().astype(np.float64)
-    err_o = np.abs(o - ro).max()
-    assert err_o <= atol_out, f"max |out - oracle| = {err_o}"
-    assert np.array_equal(np.isneginf(l), np.isneginf(rl))
-    fin = np.isfinite(rl)
-    err_l = np.abs(l[fin] - rl[fin]).max() if fin.any() else 0.0
-    assert err_l <= atol_lse, f"max |lse - oracle| = {err_l}"
+    err_o, _, err_l = check_values(o, l, ro, rl, label, atol_out, atol_lse)
     return float(err_o), float(err_l)
 
 

@@ -23,8 +23,9 @@ def _rank_main(rank, world, port, q):
     try:
         bench.barrier(pg)
         mx = bench.max_over_ranks(10.0 + 5.0 * r, pg)       # rank-dependent "timed total"
+        passes = bench.max_over_ranks_vec([1.0 + r, 5.0 - r, 3.0], pg)   # per-pass times, element-wise
         bench.barrier(pg)
-        q.put((r, w, mx))
+        q.put((r, w, mx, tuple(passes)))
     finally:
         pg.destroy_process_group()
 
@@ -47,7 +48,7 @@ def test_two_gloo_ranks_agree_on_the_max():
         p.join(timeout=120)
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     got = sorted(q.get(timeout=5) for _ in range(2))
-    assert got == [(0, 2, 15.0), (1, 2, 15.0)]
+    assert got == [(0, 2, 15.0, (2.0, 5.0, 3.0)), (1, 2, 15.0, (2.0, 5.0, 3.0))]
 
 
 def test_world_size_must_match_gpus(monkeypatch):

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import workloads as W
-from gpu_helpers import (ATOL_LSE, ATOL_OUT, compare_full, compare_rows, covered_rows, oracle_full,
+from gpu_helpers import (ATOL_LSE, ATOL_OUT, BF16_NAN_BITS, check_values, compare_full, compare_rows, covered_rows, oracle_full,
                          plan_for, run_gpu, sample_rows, sentinel_lse, sentinel_out, to_device)
 import varlen_gqa_split_b200 as vg
 
@@ -93,8 +93,7 @@ def test_continuous_batching_one_graph_many_steps():
                                        Hq=sh.Hq, Hkv=sh.Hkv, D=sh.D)
         oc = out.cpu()[rows[:, 0], rows[:, 2]].float().numpy()
         lc = lse.cpu()[rows[:, 0], rows[:, 2]].numpy()
-        assert np.abs(oc - ro).max() <= ATOL_OUT, f"step {s}"
-        assert np.abs(lc - rl).max() <= ATOL_LSE, f"step {s}"
+        check_values(oc, lc, ro, rl)
     assert plan.check_error() == 0
     del graph
 
@@ -400,6 +399,38 @@ def test_device_side_errors_are_flagged_and_rows_untouched(variant):
             for r in rows:
                 written = not bool(torch.all(raw[r] == np.int16(0x7FC0)))
                 assert written == (b not in bad), (cq, ck, b)
+
+
+@pytest.mark.parametrize("variant", [MMA, TC])
+def test_bounded_wait_runs_out_and_plan_recovers(variant):
+    """A merge wait that can never be satisfied (the plan's test hook adds a
+    part nobody writes) gives up after the plan's wait limit: the call ends,
+    ATTN_DEV_ERR_TIMEOUT is reported, the rows of every cut unit keep their
+    NaN sentinels while whole units are written and exact, and after
+    attn_check_error the same plan gives the oracle's result."""
+    sh = W.Shape("stall", B=3, Hq=32, Hkv=4, D=128, max_q=1, s_max=4096)
+    # 4096 keys (64 tiles) per KV head of sequence 0 across 16 blocks of about
+    # 18 tiles each: those units are always cut; sequence 2 (one tile) never
+    batch = W.make_batch(sh, [1, 1, 1], [4096, 300, 17], seed=41, gen_device="cuda")
+    ref_o, ref_l = oracle_full(batch)
+    plan = plan_for(sh, variant=variant, ctas=16, wait_limit_us=2000, test_stall=1)
+    q, k, v, cu_q, cu_k = to_device(batch)
+    out = sentinel_out(q.shape[0], sh.Hq, sh.D)
+    lse = sentinel_lse(q.shape[0], sh.Hq)
+    plan.run(q, k, v, cu_q, cu_k, out, lse)
+    flags = plan.check_error()                    # synchronises: the call has ended
+    assert flags & vg.ATTN_DEV_ERR_TIMEOUT, flags
+    raw = out.view(torch.int16).cpu().numpy()
+    o = out.float().cpu().numpy()
+    l_ = lse.cpu().numpy()
+    untouched = np.all(raw == np.int16(BF16_NAN_BITS), axis=2)       # [T, Hq]
+    assert untouched[0].all() and np.isnan(l_[0]).all(), "a cut unit's rows were written"
+    assert not untouched[2].any(), "a whole unit was not written"
+    written = ~untouched
+    check_values(o[written], l_[written], ref_o[written], ref_l[written])
+    # the same plan, next call: counters reset, hook cleared
+    out2, lse2 = run_gpu(plan, batch)
+    compare_full(out2, lse2, ref_o, ref_l, covered_rows(batch))
 
 
 def test_host_side_errors_launch_nothing():

@@ -4,10 +4,12 @@ whole device budget, or a latency-critical path where cudaMalloc could
 synchronise the device).  It keeps its scratch in a fixed array inside the
 library instead of allocating.
 
-Checked through the C ABI against the regular entry point (attn_run through a
-plan) on the same inputs, within the suite's tolerances, on two calls in a
-row (the second call finds the first call's leftovers in the shared array).
-This file is collected last so that a failure here cannot hide another test.
+Checked through the C ABI on two calls in a row (the second call finds the
+first call's leftovers in the shared array): each call against the fp64
+oracle with the suite's tolerances and sentinel rows, and against the regular
+entry point (attn_run through a plan) on the same inputs.  Further calls must
+not change the device's free memory.  This file is collected last so that a
+failure here cannot hide another test.
 """
 import ctypes
 
@@ -17,11 +19,10 @@ import torch
 
 import workloads as W
 import varlen_gqa_split_b200 as vg
+from gpu_helpers import (ATOL_LSE, ATOL_OUT, compare_full, covered_rows, oracle_full, sentinel_lse,
+                         sentinel_out, to_device)
 
 pytestmark = pytest.mark.gpu
-
-ATOL_OUT = 2e-2
-ATOL_LSE = 1e-3
 
 
 def _lib():
@@ -48,33 +49,55 @@ CASES = [
 
 
 @pytest.mark.parametrize("case", range(len(CASES)))
-def test_noalloc_matches_attn_run_twice(case):
+def test_noalloc_matches_oracle_and_attn_run_twice(case):
     sh, lq, lk = CASES[case]
     L = _lib()
     batch = W.make_batch(sh, lq, lk, seed=21 + case, gen_device="cuda")
-    q, k, v = batch.q, batch.k, batch.v
-    cu_q = torch.from_numpy(batch.cu_q).cuda()
-    cu_k = torch.from_numpy(batch.cu_k).cuda()
+    q, k, v, cu_q, cu_k = to_device(batch)
+    ref_o, ref_l = oracle_full(batch)
+    cov = covered_rows(batch)
     plan = vg.Plan(sh.B, sh.s_max, sh.Hq, sh.Hkv, sh.D, sh.max_q)
-    ref_o, ref_l = plan.run(q, k, v, cu_q, cu_k)
+    run_o, run_l = plan.run(q, k, v, cu_q, cu_k)
     torch.cuda.synchronize()
     assert plan.check_error() == 0
-    ref_o = ref_o.float().cpu().numpy()
-    ref_l = ref_l.cpu().numpy()
-    fin = np.isfinite(ref_l)
+    run_o = run_o.float().cpu().numpy()
+    run_l = run_l.cpu().numpy()
+    fin = np.isfinite(run_l)
     for call in range(2):
-        out = torch.full_like(q, float("nan"))
-        lse = torch.full((q.shape[0], sh.Hq), float("nan"), device="cuda")
+        out = sentinel_out(q.shape[0], sh.Hq, sh.D)
+        lse = sentinel_lse(q.shape[0], sh.Hq)
         rc = _noalloc(L, sh, q, k, v, cu_q, cu_k, out, lse)
         assert rc == 0, vg.strerror(rc)
         torch.cuda.synchronize()
+        compare_full(out.cpu(), lse.cpu(), ref_o, ref_l, cov)
         o = out.float().cpu().numpy()
         l_ = lse.cpu().numpy()
-        assert np.all(np.isfinite(o)), f"call {call}: unwritten or non-finite output"
-        assert np.abs(o - ref_o).max() <= ATOL_OUT, f"call {call}"
+        assert np.abs(o - run_o).max() <= ATOL_OUT, f"call {call}"
         assert np.array_equal(np.isfinite(l_), fin), f"call {call}: -inf pattern"
-        assert np.abs(l_[fin] - ref_l[fin]).max() <= ATOL_LSE, f"call {call}"
+        assert np.abs(l_[fin] - run_l[fin]).max() <= ATOL_LSE, f"call {call}"
     plan.close()
+
+
+def test_noalloc_calls_leave_free_memory_unchanged():
+    """After a first call (which looks up the array and, under lazy module
+    loading, commits it), further calls allocate nothing: the device's free
+    memory is the same before and after them."""
+    sh, lq, lk = CASES[0]
+    L = _lib()
+    batch = W.make_batch(sh, lq, lk, seed=31, gen_device="cuda")
+    q, k, v, cu_q, cu_k = to_device(batch)
+    out = sentinel_out(q.shape[0], sh.Hq, sh.D)
+    lse = sentinel_lse(q.shape[0], sh.Hq)
+    assert _noalloc(L, sh, q, k, v, cu_q, cu_k, out, lse) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(10):
+        assert _noalloc(L, sh, q, k, v, cu_q, cu_k, out, lse) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    ref_o, ref_l = oracle_full(batch)
+    compare_full(out.cpu(), lse.cpu(), ref_o, ref_l, covered_rows(batch))
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():

@@ -33,7 +33,7 @@ EXPORTED = ("attn_plan", "attn_plan_ex", "attn_plan_info", "attn_run", "attn_run
 class Overrides(ctypes.Structure):
     _fields_ = [("nsplit", ctypes.c_int), ("block_n", ctypes.c_int), ("variant", ctypes.c_int),
                 ("stages", ctypes.c_int), ("combine", ctypes.c_int), ("ctas", ctypes.c_int),
-                ("deterministic", ctypes.c_int)]
+                ("deterministic", ctypes.c_int), ("wait_limit_us", ctypes.c_int), ("test_stall", ctypes.c_int)]
 
 
 class PlanDesc(ctypes.Structure):
@@ -138,17 +138,19 @@ class Plan:
     """A plan: launch shape, split count and scratch fixed from constants.
 
     Plan(B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
-    stages=0, combine=0, ctas=0, deterministic=0) -- the keyword choices
-    override the planner (0 = its own; deterministic=1 asks for static tile
-    shares, -1 for run-time balancing of shared units)."""
+    stages=0, combine=0, ctas=0, deterministic=0, wait_limit_us=0, test_stall=0) -- the
+    keyword choices override the planner (0 = its own; deterministic=1 asks
+    for static tile shares, -1 for run-time balancing of shared units;
+    wait_limit_us bounds one device wait; test_stall=1 is the test hook of
+    attn_overrides that makes the first call's merge waits run out)."""
 
     def __init__(self, B_max, s_max, Hq, Hkv, D, max_q=1, *, nsplit=0, block_n=0, variant=0,
-                 stages=0, combine=0, ctas=0, deterministic=0):
+                 stages=0, combine=0, ctas=0, deterministic=0, wait_limit_us=0, test_stall=0):
         L = lib()
         h = ctypes.c_void_p()
-        if nsplit or block_n or variant or stages or combine or ctas or deterministic:
+        if nsplit or block_n or variant or stages or combine or ctas or deterministic or wait_limit_us or test_stall:
             o = Overrides(int(nsplit), int(block_n), int(variant), int(stages), int(combine), int(ctas),
-                          int(deterministic))
+                          int(deterministic), int(wait_limit_us), int(test_stall))
             rc = L.attn_plan_ex(ctypes.byref(h), int(B_max), int(s_max), int(Hq), int(Hkv), int(D),
                                 int(max_q), ctypes.byref(o))
         else:

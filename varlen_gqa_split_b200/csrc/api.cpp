@@ -38,6 +38,7 @@ struct attn_plan_s {
     int max_rt;                // tensor-core path: row tiles per sequence at most
     float *o_part;
     float2 *ml_part;
+    unsigned long long wait_ns; // limit of one bounded wait in the kernels
 };
 
 namespace {
@@ -226,6 +227,8 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     if (o && (o->nsplit < 0 || o->stages < 0 || o->ctas < 0)) return ATTN_E_INVALID_ARG;
     if (o && o->combine && o->combine != ATTN_COMBINE_KERNEL && o->combine != ATTN_COMBINE_FUSED)
         return ATTN_E_INVALID_ARG;
+    if (o && (o->wait_limit_us < 0 || o->test_stall < 0 || o->test_stall > 1)) return ATTN_E_INVALID_ARG;
+    if (o && o->test_stall && variant == ATTN_VARIANT_SIMT) return ATTN_E_UNSUPPORTED;
     d.variant = variant;
     const int tiles_max = (s_max + 63) / 64;
 
@@ -340,6 +343,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     p->qtile = qtile;
     p->max_rt = max_rt;
     p->scale_log2 = (float)((1.0 / std::sqrt((double)D)) * 1.4426950408889634);
+    p->wait_ns = o && o->wait_limit_us > 0 ? (unsigned long long)o->wait_limit_us * 1000ull : kDefaultWaitNs;
     if (cudaMalloc(&p->scratch, total) != cudaSuccess) {
         cudaGetLastError();
         delete p;
@@ -350,7 +354,12 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     p->ticket_bytes = n_ticket * sizeof(uint32_t);
     p->o_part = n_part ? reinterpret_cast<float *>(static_cast<char *>(p->scratch) + off_o) : nullptr;
     p->ml_part = n_part ? reinterpret_cast<float2 *>(static_cast<char *>(p->scratch) + off_ml) : nullptr;
-    if (cudaMemset(p->scratch, 0, off_o) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    // error word, then the test hook's stall count (parts that never arrive,
+    // cleared by attn_check_error), then the merge counters
+    const uint32_t stall = o ? (uint32_t)o->test_stall : 0u;
+    if (cudaMemset(p->scratch, 0, off_o) != cudaSuccess ||
+        cudaMemcpy(p->err + 1, &stall, sizeof(stall), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
         cudaFree(p->scratch);
         delete p;
         return ATTN_E_CUDA;
@@ -434,6 +443,8 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     p.o_part = plan->o_part;
     p.ml_part = plan->ml_part;
     p.err = plan->err;
+    p.stall = plan->err + 1;
+    p.wait_ns = plan->wait_ns;
     p.B_max = d.B_max;
     p.s_max = d.s_max;
     p.Hq = d.Hq;
@@ -578,7 +589,8 @@ ATTN_EXPORT int attn_check_error(attn_plan_t plan, void *stream, uint32_t *flags
     uint32_t h = 0;
     if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_E_CUDA;
     if (cudaMemcpy(&h, plan->err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_E_CUDA;
-    if (cudaMemset(plan->err, 0, sizeof(uint32_t)) != cudaSuccess) return ATTN_E_CUDA;
+    // the error word and the test hook's stall count
+    if (cudaMemset(plan->err, 0, 2 * sizeof(uint32_t)) != cudaSuccess) return ATTN_E_CUDA;
     // a call that stopped early may have left merge tickets part-counted
     if (h && plan->ticket_bytes && cudaMemset(plan->ticket, 0, plan->ticket_bytes) != cudaSuccess)
         return ATTN_E_CUDA;

@@ -87,14 +87,15 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
     for (int j = tid; j < n; j += kT) slots[j] = slot_of(c_first + j, seg.Pu, T, Ce);
 
     // wait for the unit's n parts, each published by done_per_part release
-    // adds (the acquire pairs with them)
-    const uint32_t parts_done = (uint32_t)(n * p.done_per_part);
+    // adds (the acquire pairs with them); p.stall adds parts that never come
+    // (a test hook, 0 otherwise), so that the bounded wait below runs out
+    const uint32_t parts_done = (uint32_t)(n * p.done_per_part) + __ldg(p.stall);
     if (tid == 0) {
         int ok = 1;
         if (ld_acquire_gpu(p.done + u) < parts_done) {
             const unsigned long long t0 = globaltimer();
             while (ld_acquire_gpu(p.done + u) < parts_done) {
-                if (globaltimer() - t0 > kWaitLimitNs) {
+                if (globaltimer() - t0 > p.wait_ns) {
                     atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
                     ok = 0;
                     break;

@@ -18,10 +18,12 @@ namespace vgqa {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Upper bound on one pipeline wait, in nanoseconds of %globaltimer.  A healthy
-// wait lasts microseconds; past this the kernel records ATTN_DEV_ERR_TIMEOUT
-// and leaves instead of spinning forever.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Default upper bound on one wait, in nanoseconds of %globaltimer (a plan may
+// set another in Params::wait_ns).  A healthy wait lasts microseconds; past
+// the bound the kernel records ATTN_DEV_ERR_TIMEOUT and leaves instead of
+// spinning forever.  Drains (a block waiting for its own copies in flight
+// before it exits) always use this default.
+constexpr unsigned long long kWaitLimitNs = kDefaultWaitNs;
 
 // Index of the partial state of query row (b, qi, h) for split z.
 __device__ __forceinline__ long long part_index(const Params &p, int b, int qi, int h, int z) {
@@ -155,13 +157,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Bounded: returns
-// false after kWaitLimitNs (the caller then records ATTN_DEV_ERR_TIMEOUT and
+// false after limit_ns (the caller then records ATTN_DEV_ERR_TIMEOUT and
 // unwinds).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer() - t0 > kWaitLimitNs) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
     }
     return true;
 }

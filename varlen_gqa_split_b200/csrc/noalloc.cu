@@ -20,7 +20,10 @@
 // symbol, so the host never passes it to a kernel: the first call on each
 // device looks up the device address with cudaGetSymbolAddress (with that
 // device current) and caches it.  That first call also sets the kernel's
-// shared-memory attribute, so make it before any stream capture begins.
+// shared-memory attribute, so make it before any stream capture begins.  Under
+// lazy module loading (CUDA's default since 12.2) the array's memory is
+// committed on that first call, so a caller whose pool reserves the device
+// should make it before the pool does.
 //
 // Every call on a device shares the one array and leaves its contents
 // behind; each call clears the error word and the merge tickets (the parts
@@ -154,6 +157,7 @@ ATTN_EXPORT int attn_run_noalloc(int B_max, int s_max, int Hq, int Hkv, int D, i
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.lse = lse;
     p.err = reinterpret_cast<uint32_t *>(s.scratch);
+    p.wait_ns = kDefaultWaitNs;
     p.ticket = n_ticket ? reinterpret_cast<uint32_t *>(s.scratch + off_t) : nullptr;
     p.o_part = n_part ? reinterpret_cast<float *>(s.scratch + off_o) : nullptr;
     p.ml_part = n_part ? reinterpret_cast<float2 *>(s.scratch + off_ml) : nullptr;

@@ -7,6 +7,9 @@
 
 namespace vgqa {
 
+// Default upper bound on one bounded wait, in nanoseconds of %globaltimer.
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
 // Everything a split / combine launch needs.  Passed by value.
 struct Params {
     const __nv_bfloat16 *q;    // [T_q, Hq, D]
@@ -49,6 +52,9 @@ struct Params {
     long long page_stride;     // elements between consecutive pages of k and v
     int page_rows;             // page_stride / token stride when whole (tensor maps index rows
                                // page * page_rows + slot), else 0 (tensor maps index (slot, page))
+    unsigned long long wait_ns; // limit of one bounded wait on another role or block (%globaltimer ns)
+    const uint32_t *stall;     // [1] parts every cut unit's merge waits for beyond its own (0 except
+                               // under the plan's test hook, whose parts never arrive)
 };
 
 }  // namespace vgqa

@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             uint32_t phase = 0;
             // take the next free stage; false if the wait gave up
             auto acquire = [&]() -> bool {
-                const bool w = issued < stages || mbar_wait(&empty[s], phase ^ 1);
+                const bool w = issued < stages || mbar_wait(&empty[s], phase ^ 1, p.wait_ns);
                 if (__all_sync(wmask, w)) return true;
                 if (leader) atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
                 return false;
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
             for (int nt = 0; nt < NT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
 
         while (ok_run) {
-            if (!mbar_wait(&full[s], phase)) {
+            if (!mbar_wait(&full[s], phase, p.wait_ns)) {
                 atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
                 ok_run = false;
                 break;

@@ -91,7 +91,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     const unsigned long long t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
         if (*stop) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > p.wait_ns) {
             atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
             *stop = 1;
             return false;
