@@ -425,8 +425,12 @@ def test_bounded_wait_runs_out_and_plan_recovers(variant):
     l_ = lse.cpu().numpy()
     untouched = np.all(raw == np.int16(BF16_NAN_BITS), axis=2)       # [T, Hq]
     assert untouched[0].all() and np.isnan(l_[0]).all(), "a cut unit's rows were written"
-    assert not untouched[2].any(), "a whole unit was not written"
     written = ~untouched
+    # 8 short units (about 2.4 blocks' shares) meet at most 3 share boundaries:
+    # most of them are whole, written by the split kernel alone
+    assert written[1:].sum() >= 5 * sh.Hq // sh.Hkv, "whole units were not written"
+    if variant == MMA:
+        assert written[2].all()          # one-tile units, and no fixed cost per unit here: never cut
     check_values(o[written], l_[written], ref_o[written], ref_l[written])
     # the same plan, next call: counters reset, hook cleared
     out2, lse2 = run_gpu(plan, batch)
