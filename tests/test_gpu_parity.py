@@ -366,6 +366,8 @@ def test_plan_choices_follow_the_split_rule():
     assert ragged_simt.info["scratch_bytes"] <= 1024
     sq = plan_for(W.SHAPES["shortq"])
     assert sq.info["variant"] == TC and sq.info["rows_per_block"] == 128
+    tiny = plan_for(W.SHAPES["tiny"])                 # units of <= 2 tiles: one block each, none cut
+    assert tiny.info["variant"] == MMA and tiny.info["ctas"] == 2
 
 
 # ------------------------------------------------------------ errors

@@ -9,38 +9,48 @@
 // the G query heads times the q_len query tokens of a unit form the M = 128
 // side of real tensor-core tiles (kernbench2 docs/adr-proposed commit log,
 // GQA entry: G folded into the matmul M dimension; every K/V byte is read
-// once per KV head):
-//     S [128 rows x 64 keys]  = Q [128 x D] . K^T            (tcgen05.mma, S in tensor memory)
-//     O [128 rows x D]       += P [128 x 64 keys] . V        (P bf16 and O in tensor memory)
+// once per KV head).  A pipeline stage holds two of the schedule's 64-key
+// tiles of one unit (128 keys), so that both products run as wide
+// instructions and every barrier round trip is paid once per 128 keys:
+//     S [128 rows x 128 keys] = Q [128 x D] . K^T     (tcgen05.mma, Q and S in tensor memory)
+//     O [128 rows x D]       += P [128 x 128 keys] . V (P bf16 and O in tensor memory)
+// A stage whose second tile is absent (the end of a block's part of a unit)
+// runs S with N = 64 and the product over its 64 keys only.
+//
+// Tensor memory (512 columns): S in two buffers of 128 columns, O (D
+// columns), the unit's Q (D / 2 columns of bf16 pairs) and P (64 columns of
+// bf16 pairs).  Q is read from tensor memory by the first product, so the
+// tensor core reads only K from shared memory for it.
 //
 // Warp roles (320 threads):
 //   warp 9 -- producer (the whole warp walks the schedule in step, each lane
-//     issuing one box, lane 0 taking claims and stage bookkeeping): loads each
-//     unit's Q tile (one TMA box of G
-//     heads x qtile tokens, right-aligned so it ends at the row tile's last
-//     query token; rows past the sequence's own tokens are never written)
-//     into one of two Q buffers, then streams the unit's K and V tiles into a
-//     ring of shared-memory stages exactly like the warp-MMA kernel;
-//   warp 8, one lane -- MMA issuer: S(j) = Q K_j^T into one of two S buffers,
-//     then O += P(j-1) V_{j-1}, so the softmax of tile j overlaps the second
-//     product of tile j-1 (a unit's last tile is not held back: its second
-//     product follows at once); completion is tracked with tcgen05.commit on
-//     mbarriers; the warp also allocates and frees the tensor memory;
+//     issuing one box, lane 0 taking claims and stage bookkeeping): for each
+//     unit it loads the unit's Q tile into a ring stage (one TMA box per
+//     D-half of G heads x qtile tokens, right-aligned so it ends at the row
+//     tile's last query token; rows past the sequence's own tokens are never
+//     written), then pairs the unit's K and V tiles into 128-key stages;
+//   warp 8, one lane -- MMA issuer: S(j) = Q K_j^T into one of two S
+//     buffers, then O += P(j-1) V_{j-1}, so the softmax of stage j overlaps
+//     the second product of stage j-1 (a unit's last stage is not held back:
+//     its second product follows at once); completion is tracked with
+//     tcgen05.commit on mbarriers; the warp also allocates and frees the
+//     tensor memory;
 //   warps 0-7 -- softmax and epilogue.  Warp w reads tensor-memory lanes
-//     32 (w mod 4) .. +31, one query row per thread, and column half
-//     h = w / 4 of every tile (keys 32h .. 32h+31).  Each half runs its own
-//     online softmax in base-2 units over its keys and accumulates its own
-//     O_h (the product P[:, half h] V[half h] goes to a separate tensor-memory
-//     accumulator), so the two warps of a row never synchronise per tile;
-//     the epilogue merges the two halves like two split-KV partials.  The
-//     scores are masked (keys before the tile's own start when the tile was
-//     right-aligned, and keys past Lk - Lq + qi under the tail-aligned causal
-//     mask), and P is written as bf16 pairs into one of two P buffers in
-//     tensor memory, from where the second product reads its A operand.
+//     32 (w mod 4) .. +31, one query row per thread, and half h = w / 4 of
+//     every stage (its 64-key tile h).  The two warps of a row exchange their
+//     halves' maxima through shared memory once per stage, so both take the
+//     same running max and add into the one O accumulator; each keeps its own
+//     running sum.  The scores are masked (keys before the tile's own start
+//     when the tile was right-aligned, and keys past Lk - Lq + qi under the
+//     tail-aligned causal mask), and P is written as bf16 pairs into tensor
+//     memory, from where the second product reads its A operand.  They also
+//     copy each unit's Q from its ring stage into tensor memory (each warp its
+//     lanes and half of D), ahead of the previous unit's epilogue, and write
+//     the epilogue: each warp its half of D.
 //
-// The running max is rescaled lazily: O_h in tensor memory is multiplied by
+// The running max is rescaled lazily: O in tensor memory is multiplied by
 // 2^(m_old - m_new) only when a row's max grows by more than 2^8 (rare after
-// the first tile); otherwise the tile's weights are taken relative to the
+// the first stage); otherwise the stage's weights are taken relative to the
 // stale max, which stays exact in fp32 and keeps P below 2^8 in bf16.  The
 // partial (O, m, l) and the final normalisation use whatever reference max
 // the row ended with, so the result is the same softmax.
@@ -61,28 +71,46 @@ namespace {
 using namespace sched;
 
 constexpr int kRows = 128;                // MMA M: query rows of a unit
-constexpr int kSoftWarps = 8;             // two per tensor-memory lane quarter (column halves)
-constexpr int kEpiWarps = 4;              // the half-0 warps write the outputs
-constexpr int kMmaWarp = 8;              // sub-partition 0: its rows are the last to hold query rows
+constexpr int kSub = 2;                   // schedule tiles per pipeline stage
+constexpr int kStageKeys = kSub * kBN;    // 128 keys
+constexpr int kSoftWarps = 8;             // two per tensor-memory lane quarter (tile halves)
+constexpr int kMmaWarp = 8;               // sub-partition 0: its rows are the last to hold query rows
 constexpr int kProducerWarp = 9;
 constexpr int kThreads = 320;
-constexpr int kHalfKeys = kBN / 2;
-constexpr int kMetaLast = 1;              // stage flag: the block's last tile of the unit
+constexpr int kMetaLast = 1;              // stage flag: the block's last stage of the unit
 constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends here
+constexpr int kMetaQ = 4;                 // stage flag: the unit's Q tile
+constexpr int kMetaEnd = 8;               // stage flag: no data, the block's work ends here
+constexpr int kSegRing = 16;              // unit descriptors in flight (see UnitDesc)
 constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold (base-2 units)
-constexpr uint32_t kTmemCols = 512;       // S [0, 128), O_0 [128, 128 + D), O_1 [256, 256 + D), P [384, 448)
-constexpr uint32_t kColS = 0, kColO0 = 128, kColO1 = 256, kColP = 384;
-constexpr uint32_t kPCols = kBN / 2;      // bf16 pairs of one P buffer
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;             // S(j) in [128 (j mod 2), +128)
+constexpr uint32_t kColO = 256;           // O, D columns
+constexpr uint32_t kColQ = 384;           // Q, D / 2 columns of bf16 pairs
+constexpr uint32_t kColP = 448;           // P, 64 columns of bf16 pairs
 constexpr size_t kMinSmemBytes = 120 * 1024;
 
 template <int D>
 struct TcLayout {
     static constexpr int kHalves = D / 64;                  // 128-byte swizzle atoms per row
-    static constexpr int kKvRegion = kBN * 128;             // 64 keys x 128 B
-    static constexpr int kKvTile = kHalves * kKvRegion;     // K or V tile
+    static constexpr int kSubRows = kBN * 128;              // one 64-key tile of one atom column
+    static constexpr int kKvRegion = kStageKeys * 128;      // 128 keys x 128 B
+    static constexpr int kKvTile = kHalves * kKvRegion;     // K or V of a stage
     static constexpr int kStage = 2 * kKvTile;              // K + V
     static constexpr int kQRegion = kRows * 128;            // 128 rows x 128 B
-    static constexpr int kQTile = kHalves * kQRegion;
+    static constexpr uint32_t kTileBytes = 2u * kHalves * kSubRows;   // K + V of one 64-key tile
+    static constexpr int kOCols = D / 2;                    // O columns per softmax warp
+    static constexpr int kQCols = D / 4;                    // Q columns (bf16 pairs) per softmax warp
+};
+
+// What the softmax warps need of a unit, written by the producer with the
+// unit's Q stage into a ring of kSegRing entries (entry k mod kSegRing for
+// the block's k-th unit).  The producer can run at most `stages` stages (<= 8)
+// ahead of the softmax warps and every unit takes at least two stages, so an
+// entry is rewritten only after the softmax warps have left its unit.
+struct UnitDesc {
+    int b, hk, rt, role;                  // role 0: the unit is the block's alone; 1, 2: cut (OrderedWalker)
+    int q0, Lq, Lk, pad;
 };
 
 // bounded mbarrier wait that also gives up when another role raised the stop flag
@@ -110,22 +138,22 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     using L = TcLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *ring = smem;                                    // [stages][K tile | V tile]
-    uint8_t *qbuf = ring + stages * L::kStage;               // [2][Q tile]
-    uint64_t *full = reinterpret_cast<uint64_t *>(qbuf + 2 * L::kQTile);
+    uint8_t *ring = smem;                                    // [stages][K | V], or a unit's Q tile
+    uint64_t *full = reinterpret_cast<uint64_t *>(ring + stages * L::kStage);
     uint64_t *empty = full + stages;
-    uint64_t *q_full = empty + stages;       // [2] Q tile landed
-    uint64_t *q_free = q_full + 2;           // [2] last product reading the Q tile done
-    uint64_t *s_full = q_free + 2;           // [2] S(j) computed (j mod 2)
+    uint64_t *q_tm = empty + stages;         // the unit's Q is in tensor memory
+    uint64_t *q_ack = q_tm + 1;              // the MMA issuer has taken it (Q may be replaced)
+    uint64_t *s_full = q_ack + 1;            // [2] S(j) computed (j mod 2)
     uint64_t *s_free = s_full + 2;           // [2] S(j) read by the softmax warps
     uint64_t *p_full = s_free + 2;           // [2] P(j) written
     uint64_t *o_done = p_full + 2;           // [2] O += P(j) V(j) done
-    uint64_t *o_free = o_done + 2;           // O_0, O_1 read by the epilogue
-    uint64_t *xch = o_free + 1;              // half-1 (m, l) of a unit published
-    uint64_t *drain = xch + 1;               // all issued tensor-core work done
-    int2 *meta = reinterpret_cast<int2 *>(drain + 1);                         // [stages]
-    float2 *xml = reinterpret_cast<float2 *>(meta + stages);                 // [128] half-1 (m, l)
-    long long *scan = reinterpret_cast<long long *>(xml + kRows);            // [kThreads / 32]
+    uint64_t *o_free = o_done + 2;           // O read by the epilogue
+    uint64_t *xbar = o_free + 1;             // [4] the two warps of a lane quarter exchanged a value
+    uint64_t *drain = xbar + 4;              // all issued tensor-core work done
+    int4 *meta = reinterpret_cast<int4 *>(drain + 1);                         // [stages]
+    UnitDesc *units = reinterpret_cast<UnitDesc *>(meta + stages);           // [kSegRing]
+    float *xbuf = reinterpret_cast<float *>(units + kSegRing);               // [2][2 halves][128]
+    long long *scan = reinterpret_cast<long long *>(xbuf + 4 * kRows);       // [kThreads / 32]
     long long *first = scan + kThreads / 32;                                 // [3]
     volatile int *stop = reinterpret_cast<volatile int *>(first + 3);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(first + 3) + 1;
@@ -140,18 +168,18 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kSoftWarps);   // the MMA's commit (or arrival) + each softmax warp
+            mbar_init(&empty[s], 1 + kSoftWarps);   // the MMA issuer (commit or arrival) + each softmax warp
         }
+        mbar_init(q_tm, kSoftWarps);
+        mbar_init(q_ack, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&q_full[i], 1);
-            mbar_init(&q_free[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&s_free[i], kSoftWarps);
             mbar_init(&p_full[i], kSoftWarps);
             mbar_init(&o_done[i], 1);
         }
-        mbar_init(o_free, kEpiWarps);
-        mbar_init(xch, kSoftWarps - kEpiWarps);
+        mbar_init(o_free, kSoftWarps);
+        for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
         mbar_init(drain, 1);
         *stop = 0;
         fence_barrier_init();
@@ -174,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     if constexpr (!PAGED) {
         Share sp;
         if (block_share(p, c, gridDim.x, tid, kThreads, false, scan, first, sp, true) && warp == kProducerWarp)
-            first_tiles(p, c, sp, kPrefetchBytes / L::kStage, true, [&](const Segment &sg, int t) {
+            first_tiles(p, c, sp, kPrefetchBytes / (int)L::kTileBytes, true, [&](const Segment &sg, int t) {
                 const int row = sg.s.k0 + min(t * kBN, sg.s.Lk - kBN);
 #pragma unroll
                 for (int hf = 0; hf < L::kHalves; ++hf) {
@@ -196,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     const int G = p.G, QT = p.qtile;                         // query tokens per row tile
 
     if (has_work && warp == kProducerWarp) {
+
         // ---------------------------------------------------------- producer
         // the whole warp walks the schedule in step and each lane loads one
         // box of a tile (a D-half of K or V; up to 32 boxes from small
@@ -204,8 +233,11 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         const bool leader = lane == 0;
         const uint64_t pol = l2_evict_first();
         const uint32_t q_bytes = (uint32_t)(L::kHalves * G * QT * 128);
-        int s = 0, issued = 0, k = 0;
+        int s = 0, issued = 0;
         uint32_t phase = 0;
+        int nseg = 0;                        // units begun
+        int nsub = 0;                        // tiles in the open stage (0: none open)
+        int ks_a = 0, ks_b = 0;              // key starts of the open stage's tiles
         auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
             return __all_sync(wmask, wait_bar(bar, parity, stop, p));
         };
@@ -217,32 +249,44 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 phase ^= 1;
             }
         };
-        // the stage's key start and flags, and the bytes its loads bring
-        // (before any lane issues one)
-        auto open_stage = [&](int ks, bool last) -> uint8_t * {
+        // the open stage is complete: its key starts and flags, then the
+        // arrival that lets its phase finish once its bytes have landed
+        auto close = [&](bool last) {
             if (leader) {
-                meta[s] = make_int2(ks, last ? kMetaLast : 0);
-                mbar_arrive_expect_tx(&full[s], L::kStage);
+                meta[s] = make_int4(ks_a, nsub == 2 ? ks_b : -1, last ? kMetaLast : 0, 0);
+                mbar_arrive(&full[s]);
             }
             __syncwarp(wmask);
-            return ring + s * L::kStage;
+            nsub = 0;
+            advance();
         };
-        auto begin = [&](const Segment &sg, int) -> bool {
+        auto begin = [&](const Segment &sg, int role) -> bool {
             if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk, lane, 32);
-            const int qb = k & 1;
-            if (k >= 2 && !wait_all(&q_free[qb], ((k - 2) >> 1) & 1)) return false;
+            if (!acquire()) return false;
             if (leader) {
-                mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+                UnitDesc &u = units[nseg % kSegRing];
+                u.b = sg.b;
+                u.hk = sg.hk;
+                u.rt = sg.rt;
+                u.role = role;
+                u.q0 = sg.s.q0;
+                u.Lq = sg.s.Lq;
+                u.Lk = sg.s.Lk;
+                meta[s] = make_int4(0, -1, kMetaQ, nseg);
+                mbar_arrive_expect_tx(&full[s], q_bytes);
                 // the box ends at the row tile's last query token
                 const int t_end = sg.s.q0 + sg.s.Lq - sg.rt * QT;
 #pragma unroll
                 for (int hf = 0; hf < L::kHalves; ++hf)
-                    tma_load_3d(qbuf + qb * L::kQTile + hf * L::kQRegion, &tm_q, &q_full[qb], hf * 64, sg.hk * G,
+                    tma_load_3d(ring + s * L::kStage + hf * L::kQRegion, &tm_q, &full[s], hf * 64, sg.hk * G,
                                 t_end - QT, pol);
             }
-            ++k;
+            __syncwarp(wmask);
+            advance();
+            ++nseg;
             return true;
         };
+        // one 64-key tile: the first or the second of a stage
         auto load_tile = [&](const Segment &sg, int tile, bool last) -> bool {
             const int ks = tile * kBN;
             if constexpr (PAGED) {
@@ -256,44 +300,65 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 const int key = ks + bi * p.page_box;
                 const bool in = mine && key < sg.s.Lk;
                 const int entry = in ? page_entry(p, sg.b, key) : 0;
-                if (!acquire()) return false;
-                uint8_t *st = open_stage(ks, last);
+                if (nsub == 0 && !acquire()) return false;
+                if (leader) mbar_expect_tx(&full[s], L::kTileBytes);
+                __syncwarp(wmask);
+                uint8_t *st = ring + s * L::kStage;
                 if (mine) {
                     // a box past the sequence (or a bad entry) reads page
                     // num_pages, outside the map: zeros
                     const int page = in ? page_checked(p, entry) : p.num_pages;
                     const int slot = key & ((1 << p.page_shift) - 1);       // 0 when pages are < 64 keys
-                    uint8_t *dst = st + tv * L::kKvTile + hf * L::kKvRegion + bi * p.page_box * 128;
+                    uint8_t *dst = st + tv * L::kKvTile + hf * L::kKvRegion + nsub * L::kSubRows +
+                                   bi * p.page_box * 128;
                     const CUtensorMap *map = tv ? &tm_v : &tm_k;
                     if (p.page_rows)
                         tma_load_3d(dst, map, &full[s], hf * 64, sg.hk, page * p.page_rows + slot, pol);
                     else
                         tma_load_4d(dst, map, &full[s], hf * 64, sg.hk, slot, page, pol);
                 }
-                advance();
-                return true;
+            } else {
+                if (nsub == 0 && !acquire()) return false;
+                if (leader) mbar_expect_tx(&full[s], L::kTileBytes);
+                __syncwarp(wmask);
+                const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
+                if (lane < 2 * L::kHalves) {                        // lane: (K or V, D-half)
+                    const int tv = lane / L::kHalves, hf = lane % L::kHalves;
+                    tma_load_3d(ring + s * L::kStage + tv * L::kKvTile + hf * L::kKvRegion + nsub * L::kSubRows,
+                                tv ? &tm_v : &tm_k, &full[s], hf * 64, sg.hk, row, pol);
+                }
             }
-            if (!acquire()) return false;
-            const int row = sg.s.k0 + min(ks, sg.s.Lk - kBN);
-            uint8_t *st = open_stage(ks, last);
-            if (lane < 2 * L::kHalves) {                        // lane: (K or V, D-half)
-                const int tv = lane / L::kHalves, hf = lane % L::kHalves;
-                tma_load_3d(st + tv * L::kKvTile + hf * L::kKvRegion, tv ? &tm_v : &tm_k, &full[s], hf * 64, sg.hk,
-                            row, pol);
-            }
-            advance();
+            // in run-time claims the second tile may precede the first
+            if (nsub == 0)
+                ks_a = ks;
+            else
+                ks_b = ks;
+            if (++nsub == kSub || last) close(last);
             return true;
         };
         auto empty_stage = [&](const Segment &) -> bool {
+            if (nsub) close(false);                                 // a half stage of claimed tiles
             if (!acquire()) return false;
             if (leader) {
-                meta[s] = make_int2(0, kMetaLast | kMetaEmpty);
+                meta[s] = make_int4(0, -1, kMetaLast | kMetaEmpty, 0);
                 mbar_arrive(&full[s]);
             }
+            __syncwarp(wmask);
             advance();
             return true;
         };
-        if (!feed_tiles<true>(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage)) *stop = 1;
+        bool fed = feed_tiles<true>(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage);
+        if (nsub) close(false);              // only after a stop: no stage stays without its arrival
+        // the end of the block's work, for the consumers
+        if (fed && (fed = acquire())) {
+            if (leader) {
+                meta[s] = make_int4(0, -1, kMetaEnd, 0);
+                mbar_arrive(&full[s]);
+            }
+            __syncwarp(wmask);
+            advance();
+        }
+        if (!fed) *stop = 1;
         // let the loads in flight land before the block can exit (bounded,
         // also after a stop: the copies target this block's shared memory)
         for (int i = 0; i < min(issued, stages); ++i) {
@@ -303,97 +368,98 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             }
             mbar_wait(&full[s], phase);
         }
-        if (k >= 1) mbar_wait(&q_full[(k - 1) & 1], ((k - 1) >> 1) & 1);
-        if (k >= 2) mbar_wait(&q_full[k & 1], ((k - 2) >> 1) & 1);
     } else if (has_work && warp == kMmaWarp) {
+
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t kIdS = tc::idesc_bf16_f32(kRows, kBN, false);
+            constexpr uint32_t kIdS2 = tc::idesc_bf16_f32(kRows, kStageKeys, false);
+            constexpr uint32_t kIdS1 = tc::idesc_bf16_f32(kRows, kBN, false);
             constexpr uint32_t kIdO = tc::idesc_bf16_f32(kRows, D, true);
-            const uint32_t ring0 = smem_u32(ring), q0 = smem_u32(qbuf);
+            const uint32_t ring0 = smem_u32(ring);
             int j = 0, k = 0, e = 0, s = 0;
             uint32_t sph = 0;                       // ring position and phase
             bool have_prev = false, ok = true;
-            int pj = 0, ps = 0, pe = 0;
+            int pj = 0, ps = 0, pe = 0, pn = 0;
             bool pfirst = false;
-            // O_h += P(pj)[:, half h] V(pj)[half h]: waits for the softmax
-            // warps' P and, at a unit's first tile, for the epilogue of the
+            auto next_stage = [&](int &cs, int4 &mt) -> bool {
+                if (!wait_bar(&full[s], sph, stop, p)) return false;
+                mt = meta[s];
+                cs = s;
+                if (++s == stages) {
+                    s = 0;
+                    sph ^= 1;
+                }
+                return true;
+            };
+            // O += P(pj) V(pj) over the stage's pn tiles: waits for the softmax
+            // warps' P and, at a unit's first stage, for the epilogue of the
             // previous unit
             auto issue_pv = [&]() -> bool {
                 if (!wait_bar(&p_full[pj & 1], (pj >> 1) & 1, stop, p)) return false;
                 if (pfirst && pe >= 1 && !wait_bar(o_free, (pe - 1) & 1, stop, p)) return false;
                 tc::fence_after_sync();
                 const uint64_t v0 = tc::smem_desc_sw128(ring0 + ps * L::kStage + L::kKvTile, L::kKvRegion, 1024);
-                const uint32_t pa = tmem + kColP + (pj & 1) * kPCols;
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int kk = 0; kk < kHalfKeys / 16; ++kk) {
-                        const int key = h * kHalfKeys + kk * 16;
-                        tc::mma_bf16_ts(tmem + (h ? kColO1 : kColO0), pa + key / 2, v0 + ((key * 128) >> 4), kIdO,
+                for (int kk = 0; kk < kStageKeys / 16; ++kk) {
+                    if (kk * 16 < pn * kBN)
+                        tc::mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, v0 + ((kk * 16 * 128) >> 4), kIdO,
                                         !pfirst || kk > 0);
-                    }
+                }
                 tc::commit(smem_u32(&empty[ps]));
                 tc::commit(smem_u32(&o_done[pj & 1]));
                 return true;
             };
-            OrderedWalker wk;
-            wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
-            Segment seg;
-            int role;
-            while (ok && wk.next(p, seg, role)) {
-                const int qb = k & 1;
-                if (!(ok = wait_bar(&q_full[qb], (k >> 1) & 1, stop, p))) break;
-                const uint32_t qa = q0 + qb * L::kQTile;
+            while (ok) {
+                // the unit's Q stage (the softmax warps copy it into tensor
+                // memory), or the end of the block's work
+                int cs;
+                int4 mt;
+                if (!(ok = next_stage(cs, mt))) break;
+                mbar_arrive(&empty[cs]);
+                if (mt.z & kMetaEnd) break;
+                if (!(ok = wait_bar(q_tm, k & 1, stop, p))) break;
+                mbar_arrive(q_ack);
+                ++k;
                 bool first = true;
                 while (true) {
-                    if (!(ok = wait_bar(&full[s], sph, stop, p))) break;
-                    const int2 mt = meta[s];
-                    const int cs_ = s;
-                    if (++s == stages) {
-                        s = 0;
-                        sph ^= 1;
-                    }
-                    if (mt.y & kMetaEmpty) {
+                    if (!(ok = next_stage(cs, mt))) break;
+                    if (mt.z & kMetaEmpty) {
                         // the block's part of the unit ends here: flush the
-                        // deferred product of its last tile, if any, and
-                        // free the Q buffer once the products reading it are
-                        // done (the commit tracks them)
-                        mbar_arrive(&empty[cs_]);
+                        // deferred product of its last stage, if any
+                        mbar_arrive(&empty[cs]);
                         if (have_prev) {
                             if (!(ok = issue_pv())) break;
                             have_prev = false;
                             ++e;
                         }
-                        tc::commit(smem_u32(&q_free[qb]));
                         break;
                     }
                     const int b = j & 1;
+                    const int n = mt.y >= 0 ? 2 : 1;
                     if (j >= 2 && !(ok = wait_bar(&s_free[b], ((j - 2) >> 1) & 1, stop, p))) break;
                     tc::fence_after_sync();
                     // descriptors advance by adding (byte offset >> 4) to the
                     // start-address field (shared addresses stay below 2^18)
-                    const uint64_t a0 = tc::smem_desc_sw128(qa, 16, 1024);
-                    const uint64_t b0 = tc::smem_desc_sw128(ring0 + cs_ * L::kStage, 16, 1024);
+                    const uint64_t b0 = tc::smem_desc_sw128(ring0 + cs * L::kStage, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const int hf = kk >> 2, cc = (kk & 3) * 32;
-                        tc::mma_bf16_ss(tmem + kColS + b * kBN, a0 + ((hf * L::kQRegion + cc) >> 4),
-                                        b0 + ((hf * L::kKvRegion + cc) >> 4), kIdS, kk > 0);
+                        tc::mma_bf16_ts(tmem + kColS + b * kStageKeys, tmem + kColQ + kk * 8,
+                                        b0 + ((hf * L::kKvRegion + cc) >> 4), n == 2 ? kIdS2 : kIdS1, kk > 0);
                     }
                     tc::commit(smem_u32(&s_full[b]));
-                    if (mt.y & kMetaLast) tc::commit(smem_u32(&q_free[qb]));
                     if (have_prev && !(ok = issue_pv())) break;
                     have_prev = true;
                     pj = j;
-                    ps = cs_;
+                    ps = cs;
+                    pn = n;
                     pfirst = first;
                     pe = e;
                     first = false;
                     ++j;
-                    if (mt.y & kMetaLast) {
+                    if (mt.z & kMetaLast) {
                         // the unit's last product goes out now: the epilogue
-                        // waits for it, and the next tile may be several
+                        // waits for it, and the next stage may be several
                         // (empty) units away
                         if (!(ok = issue_pv())) break;
                         have_prev = false;
@@ -401,7 +467,6 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                         break;
                     }
                 }
-                ++k;
             }
             if (ok && have_prev) ok = issue_pv();
             if (!ok) *stop = 1;
@@ -411,11 +476,12 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         }
         __syncwarp();
     } else if (has_work && warp < kSoftWarps) {
+
         // ---------------------------------------------------------- softmax + epilogue
         const int quarter = warp & 3, half = warp >> 2;
         const int r = quarter * 32 + lane;                   // query row = tensor-memory lane
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t col_o = half ? kColO1 : kColO0;
+        const uint32_t col_o = kColO + half * L::kOCols;     // this warp's columns of O
         const float cs = p.scale_log2;
         // every lane waits; the warp goes on only if all of them succeeded,
         // so the warp-collective tensor-memory accesses stay converged
@@ -423,44 +489,116 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const bool w = wait_bar(bar, parity, stop, p);
             return __all_sync(0xffffffffu, w);
         };
-        int j = 0, e = 0, s = 0;
+        int j = 0, s = 0, kq = 0, nx = 0;
         uint32_t sph = 0;                           // ring position and phase
         bool ok = true;
-        OrderedWalker wk;
-        wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi);
-        Segment seg;
-        int role;
-        while (ok && wk.next(p, seg, role)) {
-            const int Lq = seg.s.Lq, Lk = seg.s.Lk;
-            const int tq = r / G, g = r - tq * G;
-            const int qi = tq + rt_box_start(seg.s, seg.rt, QT); // this row's query token in the sequence
-            const bool valid = tq < QT && qi >= 0;
-            const int vis = valid ? Lk - Lq + qi + 1 : 0;        // keys [0, vis) visible (tail-aligned causal)
-            // a warp none of whose 32 rows is a query row of this unit only
-            // keeps the barrier protocol (its P rows feed O rows nobody reads)
-            const bool act = __any_sync(0xffffffffu, valid);
-            float m_used = -INFINITY, l = 0.f;
-            bool first = true, has_tiles = false;
-            while (true) {
-                if (!(ok = wwait(&full[s], sph))) break;
-                const int2 mt = meta[s];
-                const int ts = s;                                // this tile's stage
+        // exchange one value per row with the other warp of this lane
+        // quarter; false if the wait gave up
+        auto exchange = [&](float mine, float &theirs) -> bool {
+            float *xb = xbuf + (nx & 1) * 2 * kRows;
+            xb[half * kRows + r] = mine;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xbar[quarter]);
+            if (!wwait(&xbar[quarter], nx & 1)) return false;
+            theirs = xb[(half ^ 1) * kRows + r];
+            ++nx;
+            return true;
+        };
+        // the next stage is the next unit's Q stage or the end of the work:
+        // Q goes to tensor memory (this warp's lanes and half of D), once the
+        // MMA issuer has taken the previous unit's Q (whose products have all
+        // completed: this warp waited for each).  more: a unit follows.
+        auto copy_q = [&](bool &more) -> bool {
+            if (!wwait(&full[s], sph)) return false;
+            more = !(meta[s].z & kMetaEnd);
+            if (!more) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
                 if (++s == stages) {
                     s = 0;
                     sph ^= 1;
                 }
-                if (mt.y & kMetaEmpty) break;
+                return true;
+            }
+            if (kq >= 1 && !wwait(q_ack, (kq - 1) & 1)) return false;
+            tc::fence_after_sync();
+            const int d0 = half * (D / 2);                       // first element of this warp's part
+            const uint8_t *qrow = ring + s * L::kStage + (d0 / 64) * L::kQRegion + r * 128;
+            const int c0 = (d0 % 64) / 8;                        // first 16-byte chunk of it
+            if constexpr (L::kQCols == 32) {
+                uint32_t qv[32];
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(qrow + (((c0 + c8) ^ (r & 7)) << 4));
+                    qv[4 * c8] = x.x;
+                    qv[4 * c8 + 1] = x.y;
+                    qv[4 * c8 + 2] = x.z;
+                    qv[4 * c8 + 3] = x.w;
+                }
+                tc::st_32x32b_x32(tmem + lane_base + kColQ + half * L::kQCols, qv);
+            } else {
+                uint32_t qv[16];
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(qrow + (((c0 + c8) ^ (r & 7)) << 4));
+                    qv[4 * c8] = x.x;
+                    qv[4 * c8 + 1] = x.y;
+                    qv[4 * c8 + 2] = x.z;
+                    qv[4 * c8 + 3] = x.w;
+                }
+                tc::st_32x32b_x16(tmem + lane_base + kColQ + half * L::kQCols, qv);
+            }
+            tc::wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&empty[s]);
+                mbar_arrive(q_tm);
+            }
+            if (++s == stages) {
+                s = 0;
+                sph ^= 1;
+            }
+            ++kq;
+            return true;
+        };
+        bool more = false;
+        ok = copy_q(more);
+        while (ok && more) {
+            const UnitDesc &u = units[(kq - 1) % kSegRing];      // the unit whose Q was copied last
+            const int Lq = u.Lq, Lk = u.Lk;
+            const int tq = r / G, g = r - tq * G;
+            const int box0 = Lq - (u.rt + 1) * QT;               // the row tile's first token (may be < 0)
+            const int qi = tq + box0;                            // this row's query token in the sequence
+            const bool valid = tq < QT && qi >= 0;
+            const int vis = valid ? Lk - Lq + qi + 1 : 0;        // keys [0, vis) visible (tail-aligned causal)
+            // a lane quarter none of whose 32 rows is a query row of this
+            // unit only keeps the barrier protocol (its P rows feed O rows
+            // nobody reads); both warps of the quarter see the same rows
+            const bool act = __any_sync(0xffffffffu, valid);
+            float m_used = -INFINITY, l = 0.f;
+            bool first = true, has_tiles = false;
+            while (true) {
+                if (!(ok = wwait(&full[s], sph))) break;
+                const int4 mt = meta[s];
+                const int ts = s;                                // this stage
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (++s == stages) {
+                    s = 0;
+                    sph ^= 1;
+                }
+                if (mt.z & kMetaEmpty) break;
                 has_tiles = true;
-                if (PAGED && mt.x + kBN > Lk) {
+                const int ks = half ? mt.y : mt.x;               // this warp's tile (< 0: absent)
+                if (PAGED && ks >= 0 && ks + kBN > Lk) {
                     // paged tile past the sequence's end: zero its V rows
                     // past Lk (weight 0 times a stale non-finite value would
                     // not be 0) before this warp's P is signalled; the stage
                     // is refilled only after the product that follows
-                    const int z0 = Lk - mt.x;
-                    uint8_t *vt = ring + ts * L::kStage + L::kKvTile;
-                    for (int i = tid; i < (kBN - z0) * L::kHalves * 8; i += kSoftWarps * 32) {
+                    const int z0 = Lk - ks;
+                    uint8_t *vt = ring + ts * L::kStage + L::kKvTile + half * L::kSubRows;
+                    for (int i = lane + quarter * 32; i < (kBN - z0) * L::kHalves * 8; i += 128) {
                         const int rr = z0 + i / (L::kHalves * 8), rest = i % (L::kHalves * 8);
                         *reinterpret_cast<uint4 *>(vt + (rest >> 3) * L::kKvRegion + rr * 128 + (rest & 7) * 16) =
                             make_uint4(0u, 0u, 0u, 0u);
@@ -477,45 +615,74 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                     }
                     first = false;
                     ++j;
-                    if (mt.y & kMetaLast) break;
+                    if (mt.z & kMetaLast) break;
                     continue;
                 }
                 tc::fence_after_sync();
-                uint32_t sv[kHalfKeys];
-                tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kBN + half * kHalfKeys, sv);
-                tc::wait_ld();
+                uint32_t sv[2][32];                              // this warp's 64 scores
+                if (ks >= 0) {
+                    tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kStageKeys + half * kBN, sv[0]);
+                    tc::ld_32x32b_x32(tmem + lane_base + kColS + b * kStageKeys + half * kBN + 32, sv[1]);
+                    tc::wait_ld();
+                }
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_free[b]);
 
-                // mask and max of this half.  The scale (> 0) enters in the
-                // exp2 argument, so the raw maximum gives the scaled one; a
-                // masked score becomes -inf, whose weight is exactly 0.
-                const int ks = mt.x, ls = PAGED ? ks : min(ks, Lk - kBN);   // key of column 0
-                const int c0 = half * kHalfKeys;
-                const int lo_c = ks - ls - c0, hi_c = min(kHalfKeys, vis - ls - c0);   // visible [lo_c, hi_c)
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                if (__all_sync(0xffffffffu, lo_c <= 0 && hi_c >= kHalfKeys)) {
+                // mask and max of this warp's tile.  The scale (> 0) enters in
+                // the exp2 argument, so the raw maximum gives the scaled one;
+                // a masked score becomes -inf, whose weight is exactly 0.
+                float mx = -INFINITY;
+                bool whole_rows = true, dead = false;            // dead: this row's weights are all 0
+                if (ks >= 0) {
+                    const int ls = PAGED ? ks : min(ks, Lk - kBN);      // key of column 0
+                    // visible columns [lo_c, lo_c + width); a row past the unit's
+                    // query rows sees none
+                    const int lo_c = max(ks - ls, 0);
+                    const int width = max(min(kBN, vis - ls) - lo_c, 0);
+                    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    // A row that sees no key of this tile (past the unit's
+                    // query rows, or before its causal limit) needs no per-key
+                    // mask: its max is -inf and its weights are forced to 0
+                    // below -- unless the tile holds keys past the sequence
+                    // read from a page's stale slots, whose scores may be
+                    // non-finite.  Per-key masking only runs where some row
+                    // sees part of the tile (a sequence's last tiles).
+                    const bool stale = PAGED && ks + kBN > Lk;
+                    whole_rows = __all_sync(0xffffffffu, (lo_c == 0 && width == kBN) || (width == 0 && !stale));
+                    if (whole_rows) {
 #pragma unroll
-                    for (int cc = 0; cc < kHalfKeys; ++cc) mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(sv[cc]));
-                } else {
+                        for (int cc = 0; cc < kBN; ++cc)
+                            mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(sv[cc >> 5][cc & 31]));
+                        if (width == 0) mx4[0] = mx4[1] = mx4[2] = mx4[3] = -INFINITY;
+                        dead = width == 0;
+                    } else {
+                        // masked by selection, no branch per key
 #pragma unroll
-                    for (int cc = 0; cc < kHalfKeys; ++cc) {
-                        if (cc < lo_c || cc >= hi_c) sv[cc] = 0xff800000u;   // -inf
-                        mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(sv[cc]));
+                        for (int cc = 0; cc < kBN; ++cc) {
+                            const bool keep = (unsigned)(cc - lo_c) < (unsigned)width;
+                            const uint32_t x = keep ? sv[cc >> 5][cc & 31] : 0xff800000u;   // -inf
+                            sv[cc >> 5][cc & 31] = x;
+                            mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(x));
+                        }
                     }
+                    mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * cs;
                 }
-                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * cs;
-                const bool need = mx > m_used + kRescaleLog2;    // false while the tile has no visible key
+                float mo;
+                if (!(ok = exchange(mx, mo))) break;
+                mx = fmaxf(mx, mo);                              // the row's max over the stage
+                const bool need = mx > m_used + kRescaleLog2;    // false while the stage has no visible key
                 const float m_new = need ? mx : m_used;
+                // P(j) replaces P(j-1), and a rescale of O must follow its
+                // product: both wait for O += P(j-1) V(j-1)
+                bool waited = j == 0;
                 if (!first && __any_sync(0xffffffffu, need)) {
-                    // O_h holds P V of earlier tiles: rescale it once their
-                    // products are done
                     if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
+                    waited = true;
                     tc::fence_after_sync();
                     const float alpha = need ? ex2(m_used - m_new) : 1.f;
 #pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch) {
+                    for (int ch = 0; ch < L::kOCols / 32; ++ch) {
                         uint32_t o[32];
                         tc::ld_32x32b_x32(tmem + lane_base + col_o + ch * 32, o);
                         tc::wait_ld();
@@ -529,113 +696,111 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                     l *= ex2(m_used - m_new);                     // ex2(-inf) = 0 on the first visible key
                     m_used = m_new;
                 }
-                const float nref = m_used == -INFINITY ? 0.f : -m_used;
-                uint32_t pk[kHalfKeys / 2];
-                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (ks >= 0) {
+                    // a dead row's scores may be anything (rows past the
+                    // unit's tokens read whatever the Q tile held): its
+                    // weights come out as ex2(-inf) = 0 through the scale 0
+                    const float nref = dead ? -INFINITY : (m_used == -INFINITY ? 0.f : -m_used);
+                    const float csr = dead ? 0.f : cs;
+                    uint32_t pk[kBN / 2];
+                    float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < kHalfKeys / 2; ++i) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), cs, nref));
-                    const float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), cs, nref));
-                    l4[i & 3] += p0 + p1;
-                    pk[i] = pack_bf16x2(p0, p1);
+                    for (int i = 0; i < kBN / 2; ++i) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sv[i >> 4][(2 * i) & 31]), csr, nref));
+                        const float p1 = ex2(fmaf(__uint_as_float(sv[i >> 4][(2 * i + 1) & 31]), csr, nref));
+                        l4[i & 3] += p0 + p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                    if (!waited) {
+                        if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
+                        tc::fence_after_sync();
+                    }
+                    tc::st_32x32b_x32(tmem + lane_base + kColP + half * (kBN / 2), pk);
+                    tc::wait_st();
                 }
-                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-                // P buffer j mod 2 was last read by O += P(j-2) V(j-2), which
-                // finished before S(j) (issued after it) was signalled
-                tc::st_32x32b_x16(tmem + lane_base + kColP + b * kPCols + half * (kHalfKeys / 2), pk);
-                tc::wait_st();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[b]);
                 first = false;
                 ++j;
-                if (mt.y & kMetaLast) break;
+                if (mt.z & kMetaLast) break;
             }
             if (!ok) break;
 
+            // the next unit's Q goes to tensor memory now, so that its first
+            // product can run during this unit's epilogue
+            const int role = u.role, ub = u.b, uhk = u.hk, urt = u.rt;
+            const long long uq0 = u.q0;
+            if (!(ok = copy_q(more))) break;
+
             // ---------------- epilogue: this block's part of the unit
+            float Lt = l, M = m_used;
             if (has_tiles) {
                 if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
                 tc::fence_after_sync();
-                if (half == 1) {
-                    // publish this half's (m, l); the half-0 warp merges
-                    xml[r] = make_float2(m_used, l);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(xch);
-                    ++e;
-                    continue;
+                if (act) {
+                    float lo;
+                    if (!(ok = exchange(l, lo))) break;
+                    Lt = l + lo;
                 }
-                if (!(ok = wwait(xch, e & 1))) break;
-                ++e;
-            } else if (half == 1) {
-                continue;
-            }
-            // half-0 warps: merge the two halves and write
-            float s0 = 1.f, s1 = 0.f, M = m_used, Lt = l;
-            if (has_tiles) {
-                const float2 o1 = xml[r];
-                M = fmaxf(m_used, o1.x);
-                const float Mref = M == -INFINITY ? 0.f : M;
-                s0 = ex2(m_used - Mref);
-                s1 = ex2(o1.x - Mref);
-                Lt = l * s0 + o1.y * s1;
             }
             const bool whole = role == 0;
             const int slot = role == 1 ? 2 * c : 2 * c + 1;
-            const int pr = (qi - rt_first(seg.s, seg.rt, QT)) * G + g;   // row within the unit's partial
-            const long long tok = seg.s.q0 + qi;
-            const int h = seg.hk * G + g;
+            const int pr = (qi - max(0, box0)) * G + g;         // row within the unit's partial
+            const long long tok = uq0 + qi;
+            const int h = uhk * G + g;
             const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+            const int d0 = half * L::kOCols;                     // this warp's first column of D
             if (has_tiles) {
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < L::kOCols / 32; ++ch) {
                     if (!act) break;
-                    uint32_t o0[32], o1[32];
+                    uint32_t o[32];
                     __syncwarp();
-                    tc::ld_32x32b_x32(tmem + lane_base + kColO0 + ch * 32, o0);   // warp-collective
-                    tc::ld_32x32b_x32(tmem + lane_base + kColO1 + ch * 32, o1);
+                    tc::ld_32x32b_x32(tmem + lane_base + col_o + ch * 32, o);   // warp-collective
                     tc::wait_ld();
-                    float v[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o0[i]) * s0 + __uint_as_float(o1[i]) * s1;
                     if (!valid) {
                     } else if (whole) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D + ch * 32);
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D + d0 + ch * 32);
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             uint4 w;
-                            w.x = pack_bf16x2(v[8 * q4 + 0] * inv, v[8 * q4 + 1] * inv);
-                            w.y = pack_bf16x2(v[8 * q4 + 2] * inv, v[8 * q4 + 3] * inv);
-                            w.z = pack_bf16x2(v[8 * q4 + 4] * inv, v[8 * q4 + 5] * inv);
-                            w.w = pack_bf16x2(v[8 * q4 + 6] * inv, v[8 * q4 + 7] * inv);
+                            w.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+                            w.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+                            w.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+                            w.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
                             dst[q4] = w;
                         }
                     } else {
-                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((long long)slot * kRows + pr) * D + ch * 32);
+                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((long long)slot * kRows + pr) * D + d0 +
+                                                                 ch * 32);
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4)
-                            dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
+                                                  __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
                     }
                 }
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(o_free);
             } else if (valid && whole) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D + d0);
 #pragma unroll
-                for (int q4 = 0; q4 < D / 8; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
+                for (int q4 = 0; q4 < L::kOCols / 8; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
             }
-            if (valid) {
+            if (valid && half == 0) {
                 if (whole)
                     p.lse[tok * p.Hq + h] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
                 else
                     p.ml_part[(long long)slot * kRows + pr] = make_float2(M, Lt);
             }
-            // publish this warp's rows of the part (the combine waits for all
-            // kEpiWarps writer warps of each of the unit's n blocks)
+            // publish this warp's rows and columns of the part (the combine
+            // waits for all kSoftWarps writer warps of each of the unit's n
+            // blocks)
             if (!whole) {
                 __syncwarp();
-                if (lane == 0) red_add_release_gpu(p.done + unit_index(p, seg.b, seg.hk, seg.rt), 1u);
+                if (lane == 0) red_add_release_gpu(p.done + unit_index(p, ub, uhk, urt), 1u);
             }
         }
         if (!ok) *stop = 1;
@@ -661,10 +826,10 @@ void *tc_kernel_ptr(bool paged) {
 size_t tc_stage_bytes(int D) { return D == 64 ? TcLayout<64>::kStage : TcLayout<128>::kStage; }
 
 size_t tc_smem_need(int D, int stages) {
-    const size_t fixed = D == 64 ? 2 * TcLayout<64>::kQTile : 2 * TcLayout<128>::kQTile;
-    // 1 KB alignment slack + ring + Q tiles + barriers + meta + half-1 (m, l) + scan +
-    // (first, T) + stop flag, tmem slot
-    return 1024 + tc_stage_bytes(D) * stages + fixed + (2 * stages + 17) * 8 + stages * 8 + kRows * 8 +
+    // 1 KB alignment slack + ring + barriers (full, empty per stage; 17 more)
+    // + meta + unit descriptors + exchange buffer + scan + (first, T) + stop
+    // flag, tmem slot
+    return 1024 + tc_stage_bytes(D) * stages + (2 * stages + 17) * 8 + stages * 16 + kSegRing * 32 + 4 * kRows * 4 +
            (kThreads / 32 + 3) * 8 + 16;
 }
 
@@ -676,7 +841,7 @@ size_t tc_smem_bytes(int D, int stages) {
 }
 
 int tc_rows() { return kRows; }
-int tc_parts_per_block() { return kEpiWarps; }
+int tc_parts_per_block() { return kSoftWarps; }
 // A unit costs about three tiles' time besides its tiles (the query load, the
 // pipeline drain of its last tile and the epilogue), measured on the
 // short-query workload; the shares count it so that blocks holding many
