@@ -173,10 +173,12 @@ def test_tc_row_layouts(Hq, Hkv, D, max_q):
     lk[1] = max(1, int(lq[1]) - 1)
     sh = W.Shape("rows", B=B + 1, Hq=Hq, Hkv=Hkv, D=D, max_q=max_q, s_max=700)
     batch = W.make_batch(sh, lq, lk, seed=21, gen_device="cuda")
-    plan = plan_for(sh, variant=TC, ctas=11)
-    out, lse = run_gpu(plan, batch, extra_q_rows=3)
     ref_o, ref_l = oracle_full(batch)
-    compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
+    for combine in (vg.ATTN_COMBINE_KERNEL, vg.ATTN_COMBINE_FUSED):
+        plan = plan_for(sh, variant=TC, ctas=11, combine=combine)
+        assert plan.info["combine"] == combine
+        out, lse = run_gpu(plan, batch, extra_q_rows=3)
+        compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
 
 
 def test_variants_agree():
@@ -193,6 +195,8 @@ def test_variants_agree():
 
 
 @pytest.mark.parametrize("kw", [{"deterministic": 1}, {"variant": TC, "deterministic": 1}, {"variant": TC},
+                                {"variant": TC, "combine": vg.ATTN_COMBINE_FUSED},
+                                {"variant": TC, "combine": vg.ATTN_COMBINE_KERNEL},
                                 {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_FUSED},
                                 {"variant": SIMT, "nsplit": 8, "combine": vg.ATTN_COMBINE_KERNEL}])
 def test_repeat_runs_bitwise_equal(kw):
@@ -403,10 +407,11 @@ def test_device_side_errors_are_flagged_and_rows_untouched(variant):
                 assert written == (b not in bad), (cq, ck, b)
 
 
-@pytest.mark.parametrize("variant", [MMA, TC])
-def test_bounded_wait_runs_out_and_plan_recovers(variant):
+@pytest.mark.parametrize("variant,combine", [(MMA, 0), (TC, vg.ATTN_COMBINE_KERNEL), (TC, vg.ATTN_COMBINE_FUSED)])
+def test_bounded_wait_runs_out_and_plan_recovers(variant, combine):
     """A merge wait that can never be satisfied (the plan's test hook adds a
-    part nobody writes) gives up after the plan's wait limit: the call ends,
+    part nobody writes; the wait is the combine kernel's, or the merging
+    block's in the fused mode) gives up after the plan's wait limit: the call ends,
     ATTN_DEV_ERR_TIMEOUT is reported, the rows of every cut unit keep their
     NaN sentinels while whole units are written and exact, and after
     attn_check_error the same plan gives the oracle's result."""
@@ -415,7 +420,7 @@ def test_bounded_wait_runs_out_and_plan_recovers(variant):
     # 18 tiles each: those units are always cut; sequence 2 (one tile) never
     batch = W.make_batch(sh, [1, 1, 1], [4096, 300, 17], seed=41, gen_device="cuda")
     ref_o, ref_l = oracle_full(batch)
-    plan = plan_for(sh, variant=variant, ctas=16, wait_limit_us=2000, test_stall=1)
+    plan = plan_for(sh, variant=variant, ctas=16, wait_limit_us=2000, test_stall=1, combine=combine)
     q, k, v, cu_q, cu_k = to_device(batch)
     out = sentinel_out(q.shape[0], sh.Hq, sh.D)
     lse = sentinel_lse(q.shape[0], sh.Hq)
@@ -488,7 +493,9 @@ def test_tc_row_tiles_long_queries(Hq, Hkv, D, max_q):
     batch = W.make_batch(sh, lq, lk, seed=29, gen_device="cuda")
     ref_o, ref_l = oracle_full(batch)
     cov = covered_rows(batch)
-    for kw in ({}, {"ctas": 5}, {"ctas": 5, "deterministic": 1}, {"ctas": 5, "deterministic": -1}):
+    for kw in ({}, {"ctas": 5}, {"ctas": 5, "deterministic": 1}, {"ctas": 5, "deterministic": -1},
+               {"ctas": 5, "combine": vg.ATTN_COMBINE_KERNEL}, {"ctas": 5, "deterministic": -1,
+                                                                "combine": vg.ATTN_COMBINE_FUSED}):
         plan = plan_for(sh, **kw)
         assert plan.info["variant"] == TC, plan.info
         out, lse = run_gpu(plan, batch, extra_q_rows=2)

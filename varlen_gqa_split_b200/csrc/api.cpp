@@ -240,8 +240,8 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         // persistent: about one block per SM, each with a deep load ring; the
         // split points follow the balanced per-block shares (nsplit and chunk
         // do not apply) and the slot-parallel combine kernel merges cut units
-        if (o && (o->nsplit || o->combine == ATTN_COMBINE_FUSED)) return ATTN_E_UNSUPPORTED;
         const bool tcv = variant == ATTN_VARIANT_TC;
+        if (o && (o->nsplit || (!tcv && o->combine == ATTN_COMBINE_FUSED))) return ATTN_E_UNSUPPORTED;
         NT = rows <= 8 ? 1 : 2;
         d.block_n = mma_block_n();
         if (tcv) {
@@ -280,9 +280,18 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         // 183 -> 175 us); the override's sign picks either
         const int det_req = o ? o->deterministic : 0;
         d.deterministic = det_req > 0 ? 1 : det_req < 0 ? 0 : (tcv ? 1 : 0);
-        d.combine = ATTN_COMBINE_KERNEL;     // slot-parallel combine, programmatic dependent launch
-        d.combine_blocks = 2 * d.ctas * combine_slots_split((Hq / Hkv) * qtile, D);
-        n_ticket = 3 * (size_t)B_max * Hkv * max_rt;   // per unit: tile claims (64-bit), part count
+        // warp-MMA path: slot-parallel combine kernel, programmatic dependent
+        // launch; tcgen05 path: by default the last block of each cut unit
+        // merges it (no second kernel)
+        // (fused where queries span several row tiles: causal prefill 189 ->
+        // 176 us; with at most one row tile per sequence each block's cut
+        // units come last, the merge would land on its critical path, and
+        // the combine kernel measured faster: short query 48.7 against 53.2 us)
+        const int want = o && o->combine ? o->combine : (tcv && max_rt > 1 ? ATTN_COMBINE_FUSED : ATTN_COMBINE_KERNEL);
+        d.combine = tcv ? want : ATTN_COMBINE_KERNEL;
+        d.combine_blocks = d.combine == ATTN_COMBINE_KERNEL ? 2 * d.ctas * combine_slots_split((Hq / Hkv) * qtile, D) : 0;
+        // per unit: tile claims (64-bit), parts written, parts finished
+        n_ticket = 4 * (size_t)B_max * Hkv * max_rt;
         n_part = 2 * (size_t)d.ctas;       // two partial slots per block
         part_rows = d.rows_per_block;
         if ((tcv ? tc_prepare(D, stages, d.ctas) : mma_prepare(D, NT, stages, d.ctas)) != cudaSuccess)
@@ -479,6 +488,7 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     p.ticket = plan->ticket;
     p.claim = reinterpret_cast<unsigned long long *>(plan->ticket);
     p.done = plan->ticket + 2 * (size_t)d.B_max * d.Hkv * plan->max_rt;
+    p.tk = plan->ticket + 3 * (size_t)d.B_max * d.Hkv * plan->max_rt;
     p.fused = d.combine == ATTN_COMBINE_FUSED;
     p.merge_bytes = plan->merge_bytes;
     p.ctas_max = d.ctas;

@@ -25,13 +25,15 @@ struct Params {
     uint32_t *ticket;          // [B_max * Hkv * row_tiles] arrival counters (fused merge)
     unsigned long long *claim; // [B_max * Hkv] tile claims of cut units (tensor-core path)
     uint32_t *done;            // [B_max * Hkv] parts written / merges started per cut unit
+    uint32_t *tk;              // [B_max * Hkv * row tiles] parts finished per cut unit (tcgen05 fused merge)
     int B_max, s_max, Hq, Hkv, D, max_q, G;
     int nsplit;                // chunks per (sequence, KV head)
     int chunk;                 // keys per chunk
     int rows_per_block;        // query rows (G * tokens) per block
     int row_tiles;             // row blocks per KV head
     float scale_log2;          // (1/sqrt(D)) * log2(e)
-    int fused;                 // nsplit > 1: the last block of a unit merges it
+    int fused;                 // the last block of a unit to finish merges it (CUDA-core path with
+                               // nsplit > 1; tcgen05 path without a combine kernel)
     int merge_bytes;           // tensor-core path: shared bytes of the merge area
     int ctas_max;              // tensor-core path: blocks of the launch (merge table size)
     int dynamic;               // tensor-core path: blocks sharing a cut unit claim its tiles

@@ -82,6 +82,8 @@ constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends 
 constexpr int kMetaQ = 4;                 // stage flag: the unit's Q tile
 constexpr int kMetaEnd = 8;               // stage flag: no data, the block's work ends here
 constexpr int kSegRing = 16;              // unit descriptors in flight (see UnitDesc)
+constexpr int kMergeNo = 1, kMergeYes = 2, kMergeFailed = 3;   // fused merge: another block merges; this
+                                                               // one; this one, but a part never came
 constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold (base-2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;             // S(j) in [128 (j mod 2), +128)
@@ -110,16 +112,19 @@ struct TcLayout {
 // entry is rewritten only after the softmax warps have left its unit.
 struct UnitDesc {
     int b, hk, rt, role;                  // role 0: the unit is the block's alone; 1, 2: cut (OrderedWalker)
-    int q0, Lq, Lk, pad;
+    int q0, Lq, Lk, w;                    // w: the unit's positions in the flattened tile space
+    long long Pu;                         // global index of its first position
+    long long pad;
 };
 
 // bounded mbarrier wait that also gives up when another role raised the stop flag
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *stop, const Params &p) {
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *stop, const Params &p,
+                                         unsigned long long factor = 1) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
         if (*stop) return false;
-        if (globaltimer() - t0 > p.wait_ns) {
+        if (globaltimer() - t0 > p.wait_ns * factor) {
             atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
             *stop = 1;
             return false;
@@ -150,13 +155,15 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     uint64_t *o_free = o_done + 2;           // O read by the epilogue
     uint64_t *xbar = o_free + 1;             // [4] the two warps of a lane quarter exchanged a value
     uint64_t *drain = xbar + 4;              // all issued tensor-core work done
-    int4 *meta = reinterpret_cast<int4 *>(drain + 1);                         // [stages]
+    uint64_t *mg = drain + 1;                // [2] fused merge: the decision published; every warp has read it
+    int4 *meta = reinterpret_cast<int4 *>(mg + 2);                            // [stages]
     UnitDesc *units = reinterpret_cast<UnitDesc *>(meta + stages);           // [kSegRing]
     float *xbuf = reinterpret_cast<float *>(units + kSegRing);               // [2][2 halves][128]
     long long *scan = reinterpret_cast<long long *>(xbuf + 4 * kRows);       // [kThreads / 32]
     long long *first = scan + kThreads / 32;                                 // [3]
     volatile int *stop = reinterpret_cast<volatile int *>(first + 3);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(first + 3) + 1;
+    volatile int *xflag = reinterpret_cast<volatile int *>(first + 3) + 2;   // fused merge decision (kMerge*)
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -181,6 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         mbar_init(o_free, kSoftWarps);
         for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
         mbar_init(drain, 1);
+        mbar_init(&mg[0], 1);
+        mbar_init(&mg[1], kSoftWarps);
         *stop = 0;
         fence_barrier_init();
     }
@@ -272,6 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 u.q0 = sg.s.q0;
                 u.Lq = sg.s.Lq;
                 u.Lk = sg.s.Lk;
+                u.w = sg.w;
+                u.Pu = sg.Pu;
                 meta[s] = make_int4(0, -1, kMetaQ, nseg);
                 mbar_arrive_expect_tx(&full[s], q_bytes);
                 // the box ends at the row tile's last query token
@@ -489,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const bool w = wait_bar(bar, parity, stop, p);
             return __all_sync(0xffffffffu, w);
         };
-        int j = 0, s = 0, kq = 0, nx = 0;
+        int j = 0, s = 0, kq = 0, nx = 0, nm = 0;   // nm: cut units ended in the fused mode
         uint32_t sph = 0;                           // ring position and phase
         bool ok = true;
         // exchange one value per row with the other warp of this lane
@@ -730,8 +741,8 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
 
             // the next unit's Q goes to tensor memory now, so that its first
             // product can run during this unit's epilogue
-            const int role = u.role, ub = u.b, uhk = u.hk, urt = u.rt;
-            const long long uq0 = u.q0;
+            const int role = u.role, ub = u.b, uhk = u.hk, urt = u.rt, uw = u.w;
+            const long long uq0 = u.q0, uPu = u.Pu;
             if (!(ok = copy_q(more))) break;
 
             // ---------------- epilogue: this block's part of the unit
@@ -750,8 +761,9 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const int pr = (qi - max(0, box0)) * G + g;         // row within the unit's partial
             const long long tok = uq0 + qi;
             const int h = uhk * G + g;
-            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
             const int d0 = half * L::kOCols;                     // this warp's first column of D
+            const long long uidx = unit_index(p, ub, uhk, urt);
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
             if (has_tiles) {
 #pragma unroll
                 for (int ch = 0; ch < L::kOCols / 32; ++ch) {
@@ -789,19 +801,122 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
 #pragma unroll
                 for (int q4 = 0; q4 < L::kOCols / 8; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
             }
-            if (valid && half == 0) {
-                if (whole)
-                    p.lse[tok * p.Hq + h] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
-                else
+            if (valid) {
+                if (whole) {
+                    if (half == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
+                } else {
+                    // both warps of the row store the same (m, l), so that each
+                    // reads back its own store in a fused merge
                     p.ml_part[(long long)slot * kRows + pr] = make_float2(M, Lt);
+                }
             }
-            // publish this warp's rows and columns of the part (the combine
-            // waits for all kSoftWarps writer warps of each of the unit's n
-            // blocks)
-            if (!whole) {
+            if (whole) continue;
+            if (!p.fused) {
+                // publish this warp's rows and columns of the part: the
+                // combine kernel waits for all kSoftWarps writer warps of each
+                // of the unit's n blocks
                 __syncwarp();
-                if (lane == 0) red_add_release_gpu(p.done + unit_index(p, ub, uhk, urt), 1u);
+                if (lane == 0) red_add_release_gpu(p.done + uidx, 1u);
+                continue;
             }
+            // Fused mode: the last of the unit's n blocks to write its part
+            // merges all n parts (in block order, so the result does not
+            // depend on which block is last) and writes the output; the
+            // others publish their parts.  The ticket decides who is last;
+            // the merging block then waits (bounded) until every other part
+            // is published.
+            const int c_first = block_of(uPu, sh.T, sh.Ce);
+            const int nparts = block_of(uPu + uw - 1, sh.T, sh.Ce) - c_first + 1;
+            if (warp == 0 && lane == 0) {
+                // one decision at a time: every warp has read the previous one
+                bool okd = nm == 0 || wait_bar(&mg[1], (nm - 1) & 1, stop, p);
+                int dec = kMergeNo;
+                if (okd && atomicAdd(p.tk + uidx, 1u) == (uint32_t)(nparts - 1)) {
+                    // last: wait until every other part is published (the
+                    // release adds, kSoftWarps per part, pair with this
+                    // acquire); p.stall adds parts that never come (a test
+                    // hook, 0 otherwise)
+                    const uint32_t need = (uint32_t)((nparts - 1) * kSoftWarps) + __ldg(p.stall);
+                    dec = kMergeYes;
+                    if (ld_acquire_gpu(p.done + uidx) < need) {
+                        const unsigned long long t0 = globaltimer();
+                        while (ld_acquire_gpu(p.done + uidx) < need) {
+                            if (globaltimer() - t0 > p.wait_ns) {
+                                atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
+                                dec = kMergeFailed;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                    }
+                    if (dec == kMergeYes) {
+                        // every other part is published and no block touches
+                        // this unit's counters again in this call: reset them
+                        p.done[uidx] = 0u;
+                        p.tk[uidx] = 0u;
+                        p.claim[uidx] = 0ull;
+                    }
+                }
+                xflag[0] = okd ? dec : (int)kMergeFailed;
+                mbar_arrive(&mg[0]);
+            }
+            // (up to twice the limit: the merging block's own wait above may
+            // take the whole limit first)
+            const bool okm = wait_bar(&mg[0], nm & 1, stop, p, 2);
+            const int dec = okm ? (int)xflag[0] : (int)kMergeFailed;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mg[1]);
+            ++nm;
+            if (!(ok = __all_sync(0xffffffffu, okm))) break;
+            if (dec == kMergeNo) {
+                __syncwarp();
+                if (lane == 0) red_add_release_gpu(p.done + uidx, 1u);
+                continue;
+            }
+            // a part that never came leaves these rows unwritten (the plan's
+            // counters are then reset by attn_check_error)
+            if (dec != kMergeYes || !valid) continue;
+            float M2 = -INFINITY;
+            for (int i = 0; i < nparts; ++i) {
+                const float2 ml = __ldcg(p.ml_part + (long long)slot_of(c_first + i, uPu, sh.T, sh.Ce) * kRows + pr);
+                if (ml.y > 0.f) M2 = fmaxf(M2, ml.x);
+            }
+            const float Mref = M2 == -INFINITY ? 0.f : M2;
+            float Ltot = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < L::kOCols / 32; ++ch) {
+                float acc[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+                for (int i = 0; i < nparts; ++i) {
+                    const long long sr = (long long)slot_of(c_first + i, uPu, sh.T, sh.Ce) * kRows + pr;
+                    const float2 ml = __ldcg(p.ml_part + sr);
+                    if (!(ml.y > 0.f)) continue;
+                    const float ws = ex2(ml.x - Mref);
+                    if (ch == 0) Ltot = fmaf(ml.y, ws, Ltot);
+                    const float4 *src = reinterpret_cast<const float4 *>(p.o_part + sr * D + d0 + ch * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 x = __ldcg(src + q4);
+                        acc[4 * q4] = fmaf(x.x, ws, acc[4 * q4]);
+                        acc[4 * q4 + 1] = fmaf(x.y, ws, acc[4 * q4 + 1]);
+                        acc[4 * q4 + 2] = fmaf(x.z, ws, acc[4 * q4 + 2]);
+                        acc[4 * q4 + 3] = fmaf(x.w, ws, acc[4 * q4 + 3]);
+                    }
+                }
+                const float invt = Ltot > 0.f ? 1.f / Ltot : 0.f;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D + d0 + ch * 32);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint4 w;
+                    w.x = pack_bf16x2(acc[8 * q4 + 0] * invt, acc[8 * q4 + 1] * invt);
+                    w.y = pack_bf16x2(acc[8 * q4 + 2] * invt, acc[8 * q4 + 3] * invt);
+                    w.z = pack_bf16x2(acc[8 * q4 + 4] * invt, acc[8 * q4 + 5] * invt);
+                    w.w = pack_bf16x2(acc[8 * q4 + 6] * invt, acc[8 * q4 + 7] * invt);
+                    dst[q4] = w;
+                }
+            }
+            if (half == 0) p.lse[tok * p.Hq + h] = Ltot > 0.f ? (M2 + log2f(Ltot)) * kLn2 : -INFINITY;
         }
         if (!ok) *stop = 1;
     }
@@ -826,11 +941,11 @@ void *tc_kernel_ptr(bool paged) {
 size_t tc_stage_bytes(int D) { return D == 64 ? TcLayout<64>::kStage : TcLayout<128>::kStage; }
 
 size_t tc_smem_need(int D, int stages) {
-    // 1 KB alignment slack + ring + barriers (full, empty per stage; 17 more)
+    // 1 KB alignment slack + ring + barriers (full, empty per stage; 19 more)
     // + meta + unit descriptors + exchange buffer + scan + (first, T) + stop
-    // flag, tmem slot
-    return 1024 + tc_stage_bytes(D) * stages + (2 * stages + 17) * 8 + stages * 16 + kSegRing * 32 + 4 * kRows * 4 +
-           (kThreads / 32 + 3) * 8 + 16;
+    // flag, tmem slot, merge flags
+    return 1024 + tc_stage_bytes(D) * stages + (2 * stages + 19) * 8 + stages * 16 + kSegRing * sizeof(UnitDesc) +
+           4 * kRows * 4 + (kThreads / 32 + 3) * 8 + 32;
 }
 
 size_t tc_smem_bytes(int D, int stages) {
@@ -876,7 +991,7 @@ cudaError_t launch_split_tc(const Params &p, const CUtensorMap &tm_q, const CUte
                     const_cast<CUtensorMap *>(&tm_v), const_cast<Params *>(&p), &st};
     const bool paged = p.block_table != nullptr;
     cudaError_t e = cudaLaunchKernelExC(&cfg, p.D == 64 ? tc_kernel_ptr<64>(paged) : tc_kernel_ptr<128>(paged), args);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || p.fused) return e;      // fused: cut units are merged by their last block
     return launch_combine_slots(p, ctas, stream);
 }
 
