@@ -957,11 +957,11 @@ size_t tc_smem_bytes(int D, int stages) {
 
 int tc_rows() { return kRows; }
 int tc_parts_per_block() { return kSoftWarps; }
-// A unit costs about three tiles' time besides its tiles (the query load, the
-// pipeline drain of its last tile and the epilogue), measured on the
-// short-query workload; the shares count it so that blocks holding many
-// small units take fewer tiles.
-int tc_unit_cost() { return 3; }
+// A unit costs about five 64-key tiles' time besides its tiles (its query
+// stage, the pipeline drain of its last stage and the epilogue); the shares
+// count it so that blocks holding many small units take fewer tiles (short
+// query: 47.9 us with 3, 47.4 with 5 or 8).
+int tc_unit_cost() { return 5; }
 
 cudaError_t tc_prepare(int D, int stages, int ctas) {
     for (bool paged : {false, true}) {
