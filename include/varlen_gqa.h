@@ -76,7 +76,11 @@ extern "C" {
 /* How split partials are merged (attn_overrides.combine / attn_plan_desc.combine). */
 #define ATTN_COMBINE_AUTO 0
 #define ATTN_COMBINE_KERNEL 1  /* a second kernel merges every row                */
-#define ATTN_COMBINE_FUSED 2   /* the last block of each unit to finish merges it  */
+#define ATTN_COMBINE_FUSED 2   /* no second kernel: the block holding a cut unit's
+                                  last part merges it (tcgen05 path, static
+                                  shares only: with deterministic = -1 the plan
+                                  fails with ATTN_E_UNSUPPORTED); on the CUDA-core
+                                  path the last block of a unit to finish does  */
 
 typedef struct attn_plan_s *attn_plan_t;   /* opaque */
 

@@ -370,6 +370,14 @@ def test_plan_choices_follow_the_split_rule():
     assert ragged_simt.info["scratch_bytes"] <= 1024
     sq = plan_for(W.SHAPES["shortq"])
     assert sq.info["variant"] == TC and sq.info["rows_per_block"] == 128
+    # static shares; one row tile per sequence: the combine kernel merges
+    assert sq.info["deterministic"] == 1 and sq.info["combine"] == vg.ATTN_COMBINE_KERNEL
+    assert sq.info["combine_blocks"] > 0
+    # queries over several row tiles: each cut unit merged by the block
+    # holding its last part, no second kernel
+    pf = plan_for(W.SHAPES["prefill"])
+    assert pf.info["variant"] == TC and pf.info["combine"] == vg.ATTN_COMBINE_FUSED
+    assert pf.info["combine_blocks"] == 0
     tiny = plan_for(W.SHAPES["tiny"])                 # units of <= 2 tiles: one block each, none cut
     assert tiny.info["variant"] == MMA and tiny.info["ctas"] == 2
 
@@ -468,6 +476,8 @@ def test_host_side_errors_launch_nothing():
         vg.Plan(1, 64, 256, 1, 64, 1, variant=TC)          # G = 256 heads of one token exceed a 128-row tile
     with pytest.raises(vg.AttnError):
         vg.Plan(1, 64, 8, 1, 128, 1, variant=MMA, nsplit=2)  # split count belongs to the SIMT grid
+    with pytest.raises(vg.AttnError):                       # the fused merge needs static shares
+        vg.Plan(1, 64, 64, 8, 128, 8, variant=TC, deterministic=-1, combine=vg.ATTN_COMBINE_FUSED)
     handle = plan.handle
     plan.close()
     assert L.attn_run(handle, q.data_ptr(), k.data_ptr(), k.data_ptr(), cu.data_ptr(), cu.data_ptr(),
@@ -494,8 +504,9 @@ def test_tc_row_tiles_long_queries(Hq, Hkv, D, max_q):
     ref_o, ref_l = oracle_full(batch)
     cov = covered_rows(batch)
     for kw in ({}, {"ctas": 5}, {"ctas": 5, "deterministic": 1}, {"ctas": 5, "deterministic": -1},
-               {"ctas": 5, "combine": vg.ATTN_COMBINE_KERNEL}, {"ctas": 5, "deterministic": -1,
-                                                                "combine": vg.ATTN_COMBINE_FUSED}):
+               {"ctas": 5, "combine": vg.ATTN_COMBINE_KERNEL}, {"ctas": 5, "deterministic": 1,
+                                                                "combine": vg.ATTN_COMBINE_FUSED},
+               {"ctas": 5, "deterministic": -1, "combine": vg.ATTN_COMBINE_KERNEL}):
         plan = plan_for(sh, **kw)
         assert plan.info["variant"] == TC, plan.info
         out, lse = run_gpu(plan, batch, extra_q_rows=2)

@@ -281,17 +281,21 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         const int det_req = o ? o->deterministic : 0;
         d.deterministic = det_req > 0 ? 1 : det_req < 0 ? 0 : (tcv ? 1 : 0);
         // warp-MMA path: slot-parallel combine kernel, programmatic dependent
-        // launch; tcgen05 path: by default the last block of each cut unit
-        // merges it (no second kernel)
-        // (fused where queries span several row tiles: causal prefill 189 ->
-        // 176 us; with at most one row tile per sequence each block's cut
-        // units come last, the merge would land on its critical path, and
-        // the combine kernel measured faster: short query 48.7 against 53.2 us)
-        const int want = o && o->combine ? o->combine : (tcv && max_rt > 1 ? ATTN_COMBINE_FUSED : ATTN_COMBINE_KERNEL);
+        // launch.  tcgen05 path: where queries span several row tiles the
+        // block holding each cut unit's last part merges it (no second
+        // kernel; causal prefill 186 -> 150 us), which needs static shares;
+        // with one row tile per sequence the combine kernel (short query:
+        // 46.0 against 47.3 us fused -- a fused merge's reads of the other
+        // parts, issued while most blocks still stream, wait about 4 us in
+        // the loaded memory system, on the merging block's critical path)
+        const int want = o && o->combine ? o->combine
+                                         : (tcv && d.deterministic && max_rt > 1 ? ATTN_COMBINE_FUSED
+                                                                                  : ATTN_COMBINE_KERNEL);
         d.combine = tcv ? want : ATTN_COMBINE_KERNEL;
+        if (d.combine == ATTN_COMBINE_FUSED && !d.deterministic) return ATTN_E_UNSUPPORTED;
         d.combine_blocks = d.combine == ATTN_COMBINE_KERNEL ? 2 * d.ctas * combine_slots_split((Hq / Hkv) * qtile, D) : 0;
-        // per unit: tile claims (64-bit), parts written, parts finished
-        n_ticket = 4 * (size_t)B_max * Hkv * max_rt;
+        // per unit: tile claims (64-bit), parts written
+        n_ticket = 3 * (size_t)B_max * Hkv * max_rt;
         n_part = 2 * (size_t)d.ctas;       // two partial slots per block
         part_rows = d.rows_per_block;
         if ((tcv ? tc_prepare(D, stages, d.ctas) : mma_prepare(D, NT, stages, d.ctas)) != cudaSuccess)
@@ -488,13 +492,13 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     p.ticket = plan->ticket;
     p.claim = reinterpret_cast<unsigned long long *>(plan->ticket);
     p.done = plan->ticket + 2 * (size_t)d.B_max * d.Hkv * plan->max_rt;
-    p.tk = plan->ticket + 3 * (size_t)d.B_max * d.Hkv * plan->max_rt;
     p.fused = d.combine == ATTN_COMBINE_FUSED;
     p.merge_bytes = plan->merge_bytes;
     p.ctas_max = d.ctas;
     p.share_stride = share_stride(d.ctas);
     const bool persistent = d.variant == ATTN_VARIANT_MMA || d.variant == ATTN_VARIANT_TC;
     p.dynamic = persistent && !d.deterministic;
+    p.head_first = d.variant == ATTN_VARIANT_TC && p.fused;
     p.done_per_part = d.variant == ATTN_VARIANT_TC ? tc_parts_per_block() : 1;
     p.unit_cost = d.variant == ATTN_VARIANT_TC ? tc_unit_cost() : 0;
     p.qtile = plan->qtile;

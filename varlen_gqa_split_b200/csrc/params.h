@@ -25,18 +25,19 @@ struct Params {
     uint32_t *ticket;          // [B_max * Hkv * row_tiles] arrival counters (fused merge)
     unsigned long long *claim; // [B_max * Hkv] tile claims of cut units (tensor-core path)
     uint32_t *done;            // [B_max * Hkv] parts written / merges started per cut unit
-    uint32_t *tk;              // [B_max * Hkv * row tiles] parts finished per cut unit (tcgen05 fused merge)
     int B_max, s_max, Hq, Hkv, D, max_q, G;
     int nsplit;                // chunks per (sequence, KV head)
     int chunk;                 // keys per chunk
     int rows_per_block;        // query rows (G * tokens) per block
     int row_tiles;             // row blocks per KV head
     float scale_log2;          // (1/sqrt(D)) * log2(e)
-    int fused;                 // the last block of a unit to finish merges it (CUDA-core path with
-                               // nsplit > 1; tcgen05 path without a combine kernel)
+    int fused;                 // no combine kernel: on the CUDA-core path (nsplit > 1) the last block
+                               // of a unit to finish merges it; on the tcgen05 path the block
+                               // holding a cut unit's last part does
     int merge_bytes;           // tensor-core path: shared bytes of the merge area
     int ctas_max;              // tensor-core path: blocks of the launch (merge table size)
     int dynamic;               // tensor-core path: blocks sharing a cut unit claim its tiles
+    int head_first;            // tensor-core path: schedule order for the fused merge (OrderedWalker)
     int done_per_part;         // tensor-core path: releases on `done` per written part
     int share_stride;          // tensor-core path: block b takes share (b * share_stride) mod blocks
     int unit_cost;             // tensor-core path: tiles' worth of fixed cost per unit in the shares

@@ -163,28 +163,59 @@ struct SegWalker {
     }
 };
 
-// A block's units in processing order: the units that lie inside its share
-// (streamed and written by this block alone) first, then the unit cut at the
-// share's start (role 1, partial slot 2c), then the unit cut at its end
-// (role 2, slot 2c + 1).  Cut units come last so that every block sharing one
-// reaches it near the end of its own work, where run-time balancing can even
-// out the blocks' finishing times without delaying any block's own units.
+// A block's units in processing order.  By default: the units that lie
+// inside its share (streamed and written by this block alone) first, then
+// the unit cut at the share's start (role 1, partial slot 2c), then the unit
+// cut at its end (role 2, slot 2c + 1).  Cut units come last so that every
+// block sharing one reaches it near the end of its own work, where run-time
+// balancing can even out the blocks' finishing times without delaying any
+// block's own units.  `head_first` (static shares with the fused merge, in
+// which the block holding a cut unit's last part merges it) orders them so
+// that the merge never waits: the unit cut at the share's end first (a head
+// or middle part, which some later block merges), then the block's own
+// units, then the unit cut at its start (whose last part this block may
+// hold, the other parts having been streamed first by their blocks).
 struct OrderedWalker {
     SegWalker wk;
     Segment first_cut, last_cut;
-    bool has_first, has_last;
-    int phase;            // 0: inside units, 1: the start-cut unit, 2: the end-cut unit, 3: done
+    bool has_first, has_last, hf;
+    int phase;            // cuts last: 0 inside units, 1 start cut, 2 end cut, 3 done;
+                          // head first: 4 end cut, 0 inside units (skipping the cuts), 1 start cut, 3 done
+    long long wk_lo;
 
     __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi,
-                         bool spec = false) {
+                         bool spec = false, bool head_first = false) {
         wk.init(p, b_first, pb_first, lo, hi, spec);
         wk_lo = lo;
         has_first = has_last = false;
+        hf = head_first;
         phase = 0;
+        if (head_first) {
+            // a first pass finds the unit cut at the share's end
+            SegWalker w2 = wk;
+            Segment s;
+            while (true) {
+                const long long g0 = w2.g;
+                if (!w2.next(p, s)) break;
+                if (g0 != wk_lo && !(s.t0 == 0 && s.t1 == s.w)) {
+                    last_cut = s;
+                    has_last = true;
+                }
+            }
+            phase = 4;
+        }
     }
 
     // role: 0 = unit inside the share, 1 = cut at the share's start, 2 = cut at its end
     __device__ bool next(const Params &p, Segment &seg, int &role) {
+        if (phase == 4) {
+            phase = 0;
+            if (has_last) {
+                seg = last_cut;
+                role = 2;
+                return true;
+            }
+        }
         if (phase == 0) {
             Segment s;
             while (true) {
@@ -199,7 +230,7 @@ struct OrderedWalker {
                 if (g0 == wk_lo) {
                     first_cut = s;
                     has_first = true;
-                } else {
+                } else if (!hf) {                  // head first: given before
                     last_cut = s;
                     has_last = true;
                 }
@@ -216,7 +247,7 @@ struct OrderedWalker {
         }
         if (phase == 2) {
             phase = 3;
-            if (has_last) {
+            if (has_last && !hf) {
                 seg = last_cut;
                 role = 2;
                 return true;
@@ -224,7 +255,6 @@ struct OrderedWalker {
         }
         return false;
     }
-    long long wk_lo;
 };
 
 // block whose share [c*T/C, (c+1)*T/C) holds global tile t
@@ -287,7 +317,11 @@ __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int t
     sh.hi = share_start(c + 1, sh.T, sh.Ce);
     long long pb = my_start;
     if (sh.lo >= pb && sh.lo < pb + my) {
-        for (int b = b_lo; b < b_hi; ++b) {
+        if (b_hi - b_lo == 1) {                              // one sequence per thread: no second read
+            first[0] = b_lo;
+            first[1] = pb;
+        }
+        for (int b = b_lo; b_hi - b_lo > 1 && b < b_hi; ++b) {
             const long long w = (long long)p.Hkv * seq_len(p, b, false, spec).tpu;
             if (sh.lo < pb + w) {
                 first[0] = b;
@@ -325,7 +359,7 @@ template <bool WARP = false, class Begin, class Tile, class None>
 __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long long pb_first, long long lo,
                                            long long hi, Begin &&begin, Tile &&tile, None &&none) {
     OrderedWalker wk;
-    wk.init(p, b_first, pb_first, lo, hi);
+    wk.init(p, b_first, pb_first, lo, hi, false, p.head_first != 0);
     Segment seg;
     int role;
     while (wk.next(p, seg, role)) {
@@ -400,13 +434,13 @@ template <class Fn>
 __device__ __forceinline__ void first_tiles(const Params &p, int c, const Share &sh, int budget, bool spec,
                                             Fn &&fn) {
     OrderedWalker wk;
-    wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, spec);
+    wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, spec, p.head_first != 0);
     Segment seg;
     int role;
     const int lane = threadIdx.x & 31;
     int done = 0;
     while (done < budget && wk.next(p, seg, role)) {
-        if (role == 0) return;                         // whole units come first: the share has one
+        if (role == 0) return;                         // the share starts on a unit of its own
         const int nt = seg.nt;
         int a = 0, dir = 1, cnt;
         if (!p.dynamic) {

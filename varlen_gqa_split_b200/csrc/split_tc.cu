@@ -82,8 +82,6 @@ constexpr int kMetaEmpty = 2;             // stage flag: no data, the unit ends 
 constexpr int kMetaQ = 4;                 // stage flag: the unit's Q tile
 constexpr int kMetaEnd = 8;               // stage flag: no data, the block's work ends here
 constexpr int kSegRing = 16;              // unit descriptors in flight (see UnitDesc)
-constexpr int kMergeNo = 1, kMergeYes = 2, kMergeFailed = 3;   // fused merge: another block merges; this
-                                                               // one; this one, but a part never came
 constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold (base-2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;             // S(j) in [128 (j mod 2), +128)
@@ -155,15 +153,16 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     uint64_t *o_free = o_done + 2;           // O read by the epilogue
     uint64_t *xbar = o_free + 1;             // [4] the two warps of a lane quarter exchanged a value
     uint64_t *drain = xbar + 4;              // all issued tensor-core work done
-    uint64_t *mg = drain + 1;                // [2] fused merge: the decision published; every warp has read it
+    uint64_t *mg = drain + 1;                // fused merge: the other parts are published ([2]: alignment)
     int4 *meta = reinterpret_cast<int4 *>(mg + 2);                            // [stages]
     UnitDesc *units = reinterpret_cast<UnitDesc *>(meta + stages);           // [kSegRing]
     float *xbuf = reinterpret_cast<float *>(units + kSegRing);               // [2][2 halves][128]
-    long long *scan = reinterpret_cast<long long *>(xbuf + 4 * kRows);       // [kThreads / 32]
+    float2 *mstash = reinterpret_cast<float2 *>(xbuf + 4 * kRows);           // [kSoftWarps * 32] fused merge
+    long long *scan = reinterpret_cast<long long *>(mstash + kSoftWarps * 32); // [kThreads / 32]
     long long *first = scan + kThreads / 32;                                 // [3]
     volatile int *stop = reinterpret_cast<volatile int *>(first + 3);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(first + 3) + 1;
-    volatile int *xflag = reinterpret_cast<volatile int *>(first + 3) + 2;   // fused merge decision (kMerge*)
+    volatile int *mflag = reinterpret_cast<volatile int *>(first + 3) + 2;   // fused merge: 1 parts ready, 2 not
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -188,8 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         mbar_init(o_free, kSoftWarps);
         for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
         mbar_init(drain, 1);
-        mbar_init(&mg[0], 1);
-        mbar_init(&mg[1], kSoftWarps);
+        mbar_init(mg, 1);
         *stop = 0;
         fence_barrier_init();
     }
@@ -269,7 +267,16 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             nsub = 0;
             advance();
         };
+        long long mu = -1;                   // fused merge: the unit whose last part this block holds
+        uint32_t mneed = 0;                  // its count once every other part is published
         auto begin = [&](const Segment &sg, int role) -> bool {
+            if (p.fused && role == 1 && sg.t1 == sg.w) {
+                // the other parts publish kSoftWarps release adds each;
+                // p.stall adds parts that never come (a test hook, 0
+                // otherwise), so that the bounded wait runs out
+                mu = unit_index(p, sg.b, sg.hk, sg.rt);
+                mneed = (uint32_t)((c - block_of(sg.Pu, sh.T, sh.Ce)) * kSoftWarps) + __ldg(p.stall);
+            }
             if constexpr (PAGED) prefetch_pages(p, sg.b, sg.s.Lk, lane, 32);
             if (!acquire()) return false;
             if (leader) {
@@ -370,6 +377,37 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             advance();
         }
         if (!fed) *stop = 1;
+        // Fused merge: with its tiles all issued, the producer waits
+        // (bounded) until the other parts of the unit this block merges are
+        // published, so that the softmax warps find them ready when they
+        // reach its epilogue (the unit is the block's last: head-first
+        // order), and resets the unit's count for the next call -- no block
+        // adds to it again in this call.  A part that never came leaves the
+        // count set and the rows unwritten; attn_check_error then resets it.
+        if (mu >= 0) {
+            if (lane == 0) {
+                int res = fed ? 1 : 2;
+                if (fed && ld_acquire_gpu(p.done + mu) < mneed) {
+                    const unsigned long long t0 = globaltimer();
+                    while (ld_acquire_gpu(p.done + mu) < mneed) {
+                        if (*stop) {
+                            res = 2;
+                            break;
+                        }
+                        if (globaltimer() - t0 > p.wait_ns) {
+                            atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
+                            res = 2;
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                }
+                if (res == 1) p.done[mu] = 0u;
+                *mflag = res;
+                mbar_arrive(mg);
+            }
+            __syncwarp();
+        }
         // let the loads in flight land before the block can exit (bounded,
         // also after a stop: the copies target this block's shared memory)
         for (int i = 0; i < min(issued, stages); ++i) {
@@ -500,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const bool w = wait_bar(bar, parity, stop, p);
             return __all_sync(0xffffffffu, w);
         };
-        int j = 0, s = 0, kq = 0, nx = 0, nm = 0;   // nm: cut units ended in the fused mode
+        int j = 0, s = 0, kq = 0, nx = 0;
         uint32_t sph = 0;                           // ring position and phase
         bool ok = true;
         // exchange one value per row with the other warp of this lane
@@ -573,6 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             ++kq;
             return true;
         };
+        bool mpend = false, mhas = false;   // fused merge pending after the loop; its unit has tiles here
         bool more = false;
         ok = copy_q(more);
         while (ok && more) {
@@ -763,6 +802,23 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const int h = uhk * G + g;
             const int d0 = half * L::kOCols;                     // this warp's first column of D
             const long long uidx = unit_index(p, ub, uhk, urt);
+            if (p.fused && !whole && uPu + uw <= sh.hi) {
+                // Fused mode: this block holds the cut unit's last part (its
+                // blocks are c_first .. c in share order).  It merges the
+                // unit: its own part straight from tensor memory, the others'
+                // from their partial slots in block order, so the result does
+                // not depend on timing.  The others streamed their parts
+                // first (the share's head-first order), so they are normally
+                // published long before; the wait for them is bounded.
+                // The unit is the block's last (head-first order), so the
+                // merge runs after the loop, where the loop's state is dead;
+                // this row's (m, l) waits in shared memory.  Nothing waits
+                // for the unit's O to be released.
+                mstash[tid] = make_float2(M, Lt);
+                mpend = true;
+                mhas = has_tiles;
+                continue;
+            }
             const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
             if (has_tiles) {
 #pragma unroll
@@ -787,10 +843,14 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                     } else {
                         float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((long long)slot * kRows + pr) * D + d0 +
                                                                  ch * 32);
+                        // kept in L2: the unit's merge reads it back soon
+                        const uint64_t keep = l2_evict_last();
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4)
-                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
-                                                  __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
+                            st_keep_f4(dst + q4,
+                                       make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
+                                                   __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3])),
+                                       keep);
                     }
                 }
                 tc::fence_before_sync();
@@ -805,118 +865,135 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                 if (whole) {
                     if (half == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
                 } else {
-                    // both warps of the row store the same (m, l), so that each
-                    // reads back its own store in a fused merge
-                    p.ml_part[(long long)slot * kRows + pr] = make_float2(M, Lt);
+                    // both warps of the row hold the same (m, l)
+                    if (half == 0) st_keep_f2(p.ml_part + (long long)slot * kRows + pr, make_float2(M, Lt), l2_evict_last());
                 }
             }
             if (whole) continue;
-            if (!p.fused) {
-                // publish this warp's rows and columns of the part: the
-                // combine kernel waits for all kSoftWarps writer warps of each
-                // of the unit's n blocks
-                __syncwarp();
-                if (lane == 0) red_add_release_gpu(p.done + uidx, 1u);
-                continue;
-            }
-            // Fused mode: the last of the unit's n blocks to write its part
-            // merges all n parts (in block order, so the result does not
-            // depend on which block is last) and writes the output; the
-            // others publish their parts.  The ticket decides who is last;
-            // the merging block then waits (bounded) until every other part
-            // is published.
-            const int c_first = block_of(uPu, sh.T, sh.Ce);
-            const int nparts = block_of(uPu + uw - 1, sh.T, sh.Ce) - c_first + 1;
-            if (warp == 0 && lane == 0) {
-                // one decision at a time: every warp has read the previous one
-                bool okd = nm == 0 || wait_bar(&mg[1], (nm - 1) & 1, stop, p);
-                int dec = kMergeNo;
-                if (okd && atomicAdd(p.tk + uidx, 1u) == (uint32_t)(nparts - 1)) {
-                    // last: wait until every other part is published (the
-                    // release adds, kSoftWarps per part, pair with this
-                    // acquire); p.stall adds parts that never come (a test
-                    // hook, 0 otherwise)
-                    const uint32_t need = (uint32_t)((nparts - 1) * kSoftWarps) + __ldg(p.stall);
-                    dec = kMergeYes;
-                    if (ld_acquire_gpu(p.done + uidx) < need) {
-                        const unsigned long long t0 = globaltimer();
-                        while (ld_acquire_gpu(p.done + uidx) < need) {
-                            if (globaltimer() - t0 > p.wait_ns) {
-                                atomicOr(p.err, ATTN_DEV_ERR_TIMEOUT);
-                                dec = kMergeFailed;
-                                break;
+            // publish this warp's rows and columns of the part: the combine
+            // kernel, or in fused mode the unit's last block, waits for all
+            // kSoftWarps writer warps of each part
+            __syncwarp();
+            if (lane == 0) red_add_release_gpu(p.done + uidx, 1u);
+        }
+        if (ok && mpend) {
+            // fused merge of the unit whose last part this block holds:
+            // the last unit whose Q was copied, this thread's row of it
+            const UnitDesc &u = units[(kq - 1) % kSegRing];
+            const long long m_uPu = u.Pu;
+            const int tq = r / G, g = r - tq * G;
+            const int box0 = u.Lq - (u.rt + 1) * QT;
+            const int qi = tq + box0;
+            const bool m_valid = tq < QT && qi >= 0;
+            const bool m_act = __any_sync(0xffffffffu, m_valid);
+            const int m_pr = (qi - max(0, box0)) * G + g;
+            const long long m_tok = u.q0 + qi;
+            const int m_h = u.hk * G + g;
+            const float2 st = mstash[tid];
+            const float m_M = st.x, m_Lt = st.y;
+            const int d0 = half * L::kOCols;                     // this warp's first column of D
+            const int c_first = block_of(m_uPu, sh.T, sh.Ce);
+            const int npo = c - c_first;                     // the other parts (>= 1)
+            const bool own = mhas && m_Lt > 0.f;
+            // the producer has seen them published (schedule order makes
+            // that early); (up to twice the limit: the producer's own
+            // wait may take the whole limit first)
+            ok = __all_sync(0xffffffffu, wait_bar(mg, 0, stop, p, 2));
+            const bool got = ok && *mflag == 1;
+            if (got && m_act) {
+                // the first other part's columns and every part's (m, l),
+                // all loads in flight at once (one L2 round trip for a
+                // unit cut once); a part that saw no key (l = 0) may not
+                // have written its O, so its values are never used
+                const long long sr0 = (long long)slot_of(c_first, m_uPu, sh.T, sh.Ce) * kRows + m_pr;
+                float4 x0[L::kOCols / 4];
+                float2 ml0 = make_float2(0.f, 0.f);
+                float Mx = own ? m_M : -INFINITY;
+                if (m_valid) {
+                    ml0 = __ldcg(p.ml_part + sr0);
+                    const float4 *src = reinterpret_cast<const float4 *>(p.o_part + sr0 * D + d0);
+#pragma unroll
+                    for (int q4 = 0; q4 < L::kOCols / 4; ++q4) x0[q4] = __ldcg(src + q4);
+#pragma unroll 4
+                    for (int i = 1; i < npo; ++i) {
+                        const float2 ml =
+                            __ldcg(p.ml_part + (long long)slot_of(c_first + i, m_uPu, sh.T, sh.Ce) * kRows + m_pr);
+                        if (ml.y > 0.f) Mx = fmaxf(Mx, ml.x);
+                    }
+                    if (ml0.y > 0.f) Mx = fmaxf(Mx, ml0.x);
+                }
+                // weights relative to the largest max: own part, then
+                // the others in block order
+                const float Mref = Mx == -INFINITY ? 0.f : Mx;
+                const float so = own ? ex2(m_M - Mref) : 0.f;
+                const bool use0 = ml0.y > 0.f;
+                const float w0 = use0 ? ex2(ml0.x - Mref) : 0.f;
+                float Ltot = (own ? m_Lt * so : 0.f) + (use0 ? ml0.y * w0 : 0.f);
+                // (the tensor-memory reads are warp-collective: every lane
+                // takes them at the same point, the per-row work follows in
+                // a branch of its own)
+#pragma unroll
+                for (int ch = 0; ch < L::kOCols / 32; ++ch) {
+                    float acc[32];
+                    if (mhas) {                                      // warp-uniform
+                        uint32_t o[32];
+                        __syncwarp();
+                        tc::ld_32x32b_x32(tmem + lane_base + col_o + ch * 32, o);   // warp-collective
+                        tc::wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc[i] = own ? __uint_as_float(o[i]) * so : 0.f;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+                    }
+                    if (m_valid) {
+                        if (use0) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4) {
+                                const float4 x = x0[ch * 8 + q4];
+                                acc[4 * q4] = fmaf(x.x, w0, acc[4 * q4]);
+                                acc[4 * q4 + 1] = fmaf(x.y, w0, acc[4 * q4 + 1]);
+                                acc[4 * q4 + 2] = fmaf(x.z, w0, acc[4 * q4 + 2]);
+                                acc[4 * q4 + 3] = fmaf(x.w, w0, acc[4 * q4 + 3]);
                             }
-                            __nanosleep(64);
+                        }
+                        // a unit cut more than once: its further parts
+                        for (int i = 1; i < npo; ++i) {
+                            const long long sr = (long long)slot_of(c_first + i, m_uPu, sh.T, sh.Ce) * kRows + m_pr;
+                            const float2 ml = __ldcg(p.ml_part + sr);
+                            const float4 *src = reinterpret_cast<const float4 *>(p.o_part + sr * D + d0 + ch * 32);
+                            float4 x[8];
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4) x[q4] = __ldcg(src + q4);
+                            if (ml.y > 0.f) {
+                                const float ws = ex2(ml.x - Mref);
+                                if (ch == 0) Ltot = fmaf(ml.y, ws, Ltot);
+#pragma unroll
+                                for (int q4 = 0; q4 < 8; ++q4) {
+                                    acc[4 * q4] = fmaf(x[q4].x, ws, acc[4 * q4]);
+                                    acc[4 * q4 + 1] = fmaf(x[q4].y, ws, acc[4 * q4 + 1]);
+                                    acc[4 * q4 + 2] = fmaf(x[q4].z, ws, acc[4 * q4 + 2]);
+                                    acc[4 * q4 + 3] = fmaf(x[q4].w, ws, acc[4 * q4 + 3]);
+                                }
+                            }
+                        }
+                        // Ltot is complete after the first chunk's pass
+                        const float invt = Ltot > 0.f ? 1.f / Ltot : 0.f;
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (m_tok * p.Hq + m_h) * D + d0 + ch * 32);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 w;
+                            w.x = pack_bf16x2(acc[8 * q4 + 0] * invt, acc[8 * q4 + 1] * invt);
+                            w.y = pack_bf16x2(acc[8 * q4 + 2] * invt, acc[8 * q4 + 3] * invt);
+                            w.z = pack_bf16x2(acc[8 * q4 + 4] * invt, acc[8 * q4 + 5] * invt);
+                            w.w = pack_bf16x2(acc[8 * q4 + 6] * invt, acc[8 * q4 + 7] * invt);
+                            dst[q4] = w;
                         }
                     }
-                    if (dec == kMergeYes) {
-                        // every other part is published and no block touches
-                        // this unit's counters again in this call: reset them
-                        p.done[uidx] = 0u;
-                        p.tk[uidx] = 0u;
-                        p.claim[uidx] = 0ull;
-                    }
+                    __syncwarp();
                 }
-                xflag[0] = okd ? dec : (int)kMergeFailed;
-                mbar_arrive(&mg[0]);
+                if (m_valid && half == 0) p.lse[m_tok * p.Hq + m_h] = Ltot > 0.f ? (Mref + log2f(Ltot)) * kLn2 : -INFINITY;
             }
-            // (up to twice the limit: the merging block's own wait above may
-            // take the whole limit first)
-            const bool okm = wait_bar(&mg[0], nm & 1, stop, p, 2);
-            const int dec = okm ? (int)xflag[0] : (int)kMergeFailed;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&mg[1]);
-            ++nm;
-            if (!(ok = __all_sync(0xffffffffu, okm))) break;
-            if (dec == kMergeNo) {
-                __syncwarp();
-                if (lane == 0) red_add_release_gpu(p.done + uidx, 1u);
-                continue;
-            }
-            // a part that never came leaves these rows unwritten (the plan's
-            // counters are then reset by attn_check_error)
-            if (dec != kMergeYes || !valid) continue;
-            float M2 = -INFINITY;
-            for (int i = 0; i < nparts; ++i) {
-                const float2 ml = __ldcg(p.ml_part + (long long)slot_of(c_first + i, uPu, sh.T, sh.Ce) * kRows + pr);
-                if (ml.y > 0.f) M2 = fmaxf(M2, ml.x);
-            }
-            const float Mref = M2 == -INFINITY ? 0.f : M2;
-            float Ltot = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < L::kOCols / 32; ++ch) {
-                float acc[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-                for (int i = 0; i < nparts; ++i) {
-                    const long long sr = (long long)slot_of(c_first + i, uPu, sh.T, sh.Ce) * kRows + pr;
-                    const float2 ml = __ldcg(p.ml_part + sr);
-                    if (!(ml.y > 0.f)) continue;
-                    const float ws = ex2(ml.x - Mref);
-                    if (ch == 0) Ltot = fmaf(ml.y, ws, Ltot);
-                    const float4 *src = reinterpret_cast<const float4 *>(p.o_part + sr * D + d0 + ch * 32);
-#pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        const float4 x = __ldcg(src + q4);
-                        acc[4 * q4] = fmaf(x.x, ws, acc[4 * q4]);
-                        acc[4 * q4 + 1] = fmaf(x.y, ws, acc[4 * q4 + 1]);
-                        acc[4 * q4 + 2] = fmaf(x.z, ws, acc[4 * q4 + 2]);
-                        acc[4 * q4 + 3] = fmaf(x.w, ws, acc[4 * q4 + 3]);
-                    }
-                }
-                const float invt = Ltot > 0.f ? 1.f / Ltot : 0.f;
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (tok * p.Hq + h) * D + d0 + ch * 32);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint4 w;
-                    w.x = pack_bf16x2(acc[8 * q4 + 0] * invt, acc[8 * q4 + 1] * invt);
-                    w.y = pack_bf16x2(acc[8 * q4 + 2] * invt, acc[8 * q4 + 3] * invt);
-                    w.z = pack_bf16x2(acc[8 * q4 + 4] * invt, acc[8 * q4 + 5] * invt);
-                    w.w = pack_bf16x2(acc[8 * q4 + 6] * invt, acc[8 * q4 + 7] * invt);
-                    dst[q4] = w;
-                }
-            }
-            if (half == 0) p.lse[tok * p.Hq + h] = Ltot > 0.f ? (M2 + log2f(Ltot)) * kLn2 : -INFINITY;
         }
         if (!ok) *stop = 1;
     }
@@ -942,10 +1019,10 @@ size_t tc_stage_bytes(int D) { return D == 64 ? TcLayout<64>::kStage : TcLayout<
 
 size_t tc_smem_need(int D, int stages) {
     // 1 KB alignment slack + ring + barriers (full, empty per stage; 19 more)
-    // + meta + unit descriptors + exchange buffer + scan + (first, T) + stop
+    // + meta + unit descriptors + exchange buffer + merge stash + scan + (first, T) + stop
     // flag, tmem slot, merge flags
     return 1024 + tc_stage_bytes(D) * stages + (2 * stages + 19) * 8 + stages * 16 + kSegRing * sizeof(UnitDesc) +
-           4 * kRows * 4 + (kThreads / 32 + 3) * 8 + 32;
+           4 * kRows * 4 + kSoftWarps * 32 * 8 + (kThreads / 32 + 3) * 8 + 32;
 }
 
 size_t tc_smem_bytes(int D, int stages) {
