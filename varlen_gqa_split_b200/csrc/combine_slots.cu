@@ -27,6 +27,64 @@ namespace {
 
 using namespace sched;
 
+// Few-part merge of one unit's rows.  A pair of lanes takes 2 * NC
+// consecutive 4-column items of one row (the two lanes alternate, so each
+// 32-byte sector is read whole by one load instruction of the pair); the
+// unit's groups are split evenly over its nb combine blocks (this is block
+// bi), and a pair takes a group per step with every load of it -- the
+// row's (m, l) of each part once, and its NC items of each part -- in
+// flight at once.
+template <int D, int NP, int NC, class WriteRow>
+__device__ __forceinline__ void merge_few(const Params &p, const int *slots, int n, long long ROWS, int R, int nb,
+                                          int bi, WriteRow &&write_row) {
+    constexpr int kG = D / 4 / (2 * NC);            // groups per row
+    static_assert(kG >= 1, "a group spans at most a row");
+    const int groups = R * kG;
+    const int per = (groups + nb - 1) / nb;
+    const int g_lo = min(groups, bi * per), g_hi = min(groups, g_lo + per);
+    const int side = threadIdx.x & 1;
+    for (int gi = g_lo + (int)(threadIdx.x >> 1); gi < g_hi; gi += (int)(blockDim.x >> 1)) {
+        const int r = gi / kG, c0 = (gi % kG) * 2 * NC + side;      // this lane's first 4-column item
+        float2 ml[NP];
+        float4 o[NP][NC];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            if (j < n) {
+                const long long sr = (long long)slots[j] * ROWS + r;
+                ml[j] = __ldcg(p.ml_part + sr);
+                const float4 *src = reinterpret_cast<const float4 *>(p.o_part + sr * D) + c0;
+#pragma unroll
+                for (int q = 0; q < NC; ++q) o[j][q] = __ldcg(src + 2 * q);
+            }
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+            if (j < n && ml[j].y > 0.f) M = fmaxf(M, ml[j].x);
+        const float Mref = M == -INFINITY ? 0.f : M;
+        float L = 0.f;
+        float4 acc[NC];
+#pragma unroll
+        for (int q = 0; q < NC; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            if (j < n && ml[j].y > 0.f) {
+                const float w = ex2(ml[j].x - Mref);
+                L = fmaf(w, ml[j].y, L);
+#pragma unroll
+                for (int q = 0; q < NC; ++q) {
+                    acc[q].x = fmaf(w, o[j][q].x, acc[q].x);
+                    acc[q].y = fmaf(w, o[j][q].y, acc[q].y);
+                    acc[q].z = fmaf(w, o[j][q].z, acc[q].z);
+                    acc[q].w = fmaf(w, o[j][q].w, acc[q].w);
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < NC; ++q) write_row(r, 4 * (c0 + 2 * q), M, L, acc[q]);
+    }
+}
+
 // Combine: block 2c + k merges slice (c - c_first) of the unit block c cut at
 // its start (k = 0) or end (k = 1), if any.  The block is launched as a
 // programmatic dependent of the split kernel, so it computes the schedule
@@ -42,8 +100,7 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
     constexpr int kCols = D / 4;
     constexpr int kT = 128;
     constexpr int kBatch = 12;             // loads in flight per thread (register budget)
-    constexpr int kFewParts = 4;           // up to this many parts: item-batched merge
-    constexpr int kItems = 3;              // items per thread per pass in the item-batched merge
+    constexpr int kFewParts = 4;           // up to this many parts: row-group merge (merge_few)
     extern __shared__ __align__(16) uint8_t csm[];
     __shared__ long long scan[kT / 32];
     __shared__ long long first[3];
@@ -120,52 +177,15 @@ __global__ void __launch_bounds__(128, 4) combine_slots_kernel(const Params p, c
         if (d4 == 0) p.lse[tok * p.Hq + h] = Lt > 0.f ? (Mt + log2f(Lt)) * kLn2 : -INFINITY;
     };
     if (n <= kFewParts) {
-        // few parts: one thread per item, kItems items per pass with all
-        // their loads in flight (the merge is latency-bound)
-        const int n_items = it_hi - it_lo;
-        for (int base = 0; base < n_items; base += kT * kItems) {
-            float2 ml[kItems][kFewParts];
-            float4 o[kItems][kFewParts];
-#pragma unroll
-            for (int i = 0; i < kItems; ++i) {
-                const int w = base + i * kT + tid;
-                const int it = it_lo + (w < n_items ? w : 0);
-                const int r = it / kCols, d4 = (it % kCols) * 4;
-#pragma unroll
-                for (int j = 0; j < kFewParts; ++j) {
-                    if (j < n && w < n_items) {
-                        const long long sl = slots[j];
-                        ml[i][j] = __ldcg(p.ml_part + sl * ROWS + r);
-                        o[i][j] = __ldcg(reinterpret_cast<const float4 *>(p.o_part + (sl * ROWS + r) * D + d4));
-                    }
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < kItems; ++i) {
-                const int w = base + i * kT + tid;
-                if (w >= n_items) continue;
-                const int it = it_lo + w;
-                float M = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < kFewParts; ++j)
-                    if (j < n && ml[i][j].y > 0.f) M = fmaxf(M, ml[i][j].x);
-                const float Mref = M == -INFINITY ? 0.f : M;
-                float L = 0.f;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int j = 0; j < kFewParts; ++j) {
-                    if (j < n && ml[i][j].y > 0.f) {
-                        const float wq = ex2(ml[i][j].x - Mref);
-                        acc.x = fmaf(wq, o[i][j].x, acc.x);
-                        acc.y = fmaf(wq, o[i][j].y, acc.y);
-                        acc.z = fmaf(wq, o[i][j].z, acc.z);
-                        acc.w = fmaf(wq, o[i][j].w, acc.w);
-                        L = fmaf(wq, ml[i][j].y, L);
-                    }
-                }
-                write_row(it / kCols, (it % kCols) * 4, M, L, acc);
-            }
-        }
+        // few parts: a thread merges NC consecutive 4-column items of one row
+        // per step, with all their loads (and the row's (m, l) of each part,
+        // read once) in flight together: the merge is latency-bound, so the
+        // fewer dependent round trips the better
+        const int bi = (c - c_first) * S + sub;            // this block among the unit's nb
+        if (n <= 2)
+            merge_few<D, 2, 8>(p, slots, n, ROWS, R, nb, bi, write_row);
+        else
+            merge_few<D, kFewParts, 4>(p, slots, n, ROWS, R, nb, bi, write_row);
         __syncthreads();
         if (tid == 0 && atomicAdd(p.done + u, 1u) == parts_done + (uint32_t)(nb - 1)) p.done[u] = 0u;
         return;

@@ -175,7 +175,69 @@ struct SegWalker {
 // or middle part, which some later block merges), then the block's own
 // units, then the unit cut at its start (whose last part this block may
 // hold, the other parts having been streamed first by their blocks).
+// HF: head-first order compiled in (the tensor-core kernel); the kernels that
+// never use it keep the plain walker.
+template <bool HF = false>
 struct OrderedWalker {
+    SegWalker wk;
+    Segment first_cut, last_cut;
+    bool has_first, has_last;
+    int phase;            // 0: inside units, 1: the start-cut unit, 2: the end-cut unit, 3: done
+
+    __device__ void init(const Params &p, int b_first, long long pb_first, long long lo, long long hi,
+                         bool spec = false, bool = false) {
+        wk.init(p, b_first, pb_first, lo, hi, spec);
+        wk_lo = lo;
+        has_first = has_last = false;
+        phase = 0;
+    }
+
+    // role: 0 = unit inside the share, 1 = cut at the share's start, 2 = cut at its end
+    __device__ bool next(const Params &p, Segment &seg, int &role) {
+        if (phase == 0) {
+            Segment s;
+            while (true) {
+                const long long g0 = wk.g;
+                if (!wk.next(p, s)) break;
+                const bool whole = s.t0 == 0 && s.t1 == s.w;
+                if (whole) {
+                    seg = s;
+                    role = 0;
+                    return true;
+                }
+                if (g0 == wk_lo) {
+                    first_cut = s;
+                    has_first = true;
+                } else {
+                    last_cut = s;
+                    has_last = true;
+                }
+            }
+            phase = 1;
+        }
+        if (phase == 1) {
+            phase = 2;
+            if (has_first) {
+                seg = first_cut;
+                role = 1;
+                return true;
+            }
+        }
+        if (phase == 2) {
+            phase = 3;
+            if (has_last) {
+                seg = last_cut;
+                role = 2;
+                return true;
+            }
+        }
+        return false;
+    }
+    long long wk_lo;
+};
+
+template <>
+struct OrderedWalker<true> {
     SegWalker wk;
     Segment first_cut, last_cut;
     bool has_first, has_last, hf;
@@ -190,7 +252,7 @@ struct OrderedWalker {
         has_first = has_last = false;
         hf = head_first;
         phase = 0;
-        if (head_first) {
+        if (hf) {
             // a first pass finds the unit cut at the share's end
             SegWalker w2 = wk;
             Segment s;
@@ -355,10 +417,10 @@ __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int t
 // WARP: the whole warp calls it in step (every lane walks the same
 // schedule; lane 0 alone takes the claims and the result is broadcast), so
 // that the callbacks can spread their work over the lanes.
-template <bool WARP = false, class Begin, class Tile, class None>
+template <bool WARP = false, bool HF = false, class Begin, class Tile, class None>
 __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long long pb_first, long long lo,
                                            long long hi, Begin &&begin, Tile &&tile, None &&none) {
-    OrderedWalker wk;
+    OrderedWalker<HF> wk;
     wk.init(p, b_first, pb_first, lo, hi, false, p.head_first != 0);
     Segment seg;
     int role;
@@ -430,10 +492,10 @@ __device__ __forceinline__ bool feed_tiles(const Params &p, int b_first, long lo
 // tile 0; the others claim from the back, and together their first claims
 // take the unit's last tiles, so the j-th of them (j >= 1 in share order)
 // takes tiles [nt - j * budget, nt - (j - 1) * budget).
-template <class Fn>
+template <bool HF = false, class Fn>
 __device__ __forceinline__ void first_tiles(const Params &p, int c, const Share &sh, int budget, bool spec,
                                             Fn &&fn) {
-    OrderedWalker wk;
+    OrderedWalker<HF> wk;
     wk.init(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, spec, p.head_first != 0);
     Segment seg;
     int role;

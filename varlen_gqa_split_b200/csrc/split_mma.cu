@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
         }
     };
 
-    OrderedWalker wk;
+    OrderedWalker<> wk;
     wk.init(p, b_first, pb_first, lo, hi);
     Segment cur, nxt;
     int role_cur, role_nxt;

@@ -131,9 +131,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     return true;
 }
 
-// PAGED: K and V come from a paged cache (block table); a separate
-// instantiation keeps the packed kernel free of that code
-template <int D, bool PAGED>
+// PAGED: K and V come from a paged cache (block table); FUSED: the fused
+// merge (head-first unit order, the merge after the unit loop).  Separate
+// instantiations keep each kernel free of the code it does not run.
+template <int D, bool PAGED, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                const __grid_constant__ CUtensorMap tm_k,
                                                                const __grid_constant__ CUtensorMap tm_v,
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
     if constexpr (!PAGED) {
         Share sp;
         if (block_share(p, c, gridDim.x, tid, kThreads, false, scan, first, sp, true) && warp == kProducerWarp)
-            first_tiles(p, c, sp, kPrefetchBytes / (int)L::kTileBytes, true, [&](const Segment &sg, int t) {
+            first_tiles<FUSED>(p, c, sp, kPrefetchBytes / (int)L::kTileBytes, true, [&](const Segment &sg, int t) {
                 const int row = sg.s.k0 + min(t * kBN, sg.s.Lk - kBN);
 #pragma unroll
                 for (int hf = 0; hf < L::kHalves; ++hf) {
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
         long long mu = -1;                   // fused merge: the unit whose last part this block holds
         uint32_t mneed = 0;                  // its count once every other part is published
         auto begin = [&](const Segment &sg, int role) -> bool {
-            if (p.fused && role == 1 && sg.t1 == sg.w) {
+            if (FUSED && role == 1 && sg.t1 == sg.w) {
                 // the other parts publish kSoftWarps release adds each;
                 // p.stall adds parts that never come (a test hook, 0
                 // otherwise), so that the bounded wait runs out
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             advance();
             return true;
         };
-        bool fed = feed_tiles<true>(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage);
+        bool fed = feed_tiles<true, FUSED>(p, sh.b_first, sh.pb_first, sh.lo, sh.hi, begin, load_tile, empty_stage);
         if (nsub) close(false);              // only after a stop: no stage stays without its arrival
         // the end of the block's work, for the consumers
         if (fed && (fed = acquire())) {
@@ -802,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
             const int h = uhk * G + g;
             const int d0 = half * L::kOCols;                     // this warp's first column of D
             const long long uidx = unit_index(p, ub, uhk, urt);
-            if (p.fused && !whole && uPu + uw <= sh.hi) {
+            if (FUSED && !whole && uPu + uw <= sh.hi) {
                 // Fused mode: this block holds the cut unit's last part (its
                 // blocks are c_first .. c in share order).  It merges the
                 // unit: its own part straight from tensor memory, the others'
@@ -1008,9 +1009,12 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
 }
 
 template <int D>
-void *tc_kernel_ptr(bool paged) {
-    return paged ? reinterpret_cast<void *>(split_tc_kernel<D, true>)
-                 : reinterpret_cast<void *>(split_tc_kernel<D, false>);
+void *tc_kernel_ptr(bool paged, bool fused) {
+    if (fused)
+        return paged ? reinterpret_cast<void *>(split_tc_kernel<D, true, true>)
+                     : reinterpret_cast<void *>(split_tc_kernel<D, false, true>);
+    return paged ? reinterpret_cast<void *>(split_tc_kernel<D, true, false>)
+                 : reinterpret_cast<void *>(split_tc_kernel<D, false, false>);
 }
 
 }  // namespace
@@ -1041,12 +1045,13 @@ int tc_parts_per_block() { return kSoftWarps; }
 int tc_unit_cost() { return 5; }
 
 cudaError_t tc_prepare(int D, int stages, int ctas) {
-    for (bool paged : {false, true}) {
-        void *fn = D == 64 ? tc_kernel_ptr<64>(paged) : tc_kernel_ptr<128>(paged);
-        const cudaError_t e =
-            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(D, stages));
-        if (e != cudaSuccess) return e;
-    }
+    for (bool paged : {false, true})
+        for (bool fused : {false, true}) {
+            void *fn = D == 64 ? tc_kernel_ptr<64>(paged, fused) : tc_kernel_ptr<128>(paged, fused);
+            const cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(D, stages));
+            if (e != cudaSuccess) return e;
+        }
     return combine_slots_prepare(D, ctas);
 }
 
@@ -1067,7 +1072,9 @@ cudaError_t launch_split_tc(const Params &p, const CUtensorMap &tm_q, const CUte
     void *args[] = {const_cast<CUtensorMap *>(&tm_q), const_cast<CUtensorMap *>(&tm_k),
                     const_cast<CUtensorMap *>(&tm_v), const_cast<Params *>(&p), &st};
     const bool paged = p.block_table != nullptr;
-    cudaError_t e = cudaLaunchKernelExC(&cfg, p.D == 64 ? tc_kernel_ptr<64>(paged) : tc_kernel_ptr<128>(paged), args);
+    const bool fused = p.fused != 0;
+    cudaError_t e = cudaLaunchKernelExC(
+        &cfg, p.D == 64 ? tc_kernel_ptr<64>(paged, fused) : tc_kernel_ptr<128>(paged, fused), args);
     if (e != cudaSuccess || p.fused) return e;      // fused: cut units are merged by their last block
     return launch_combine_slots(p, ctas, stream);
 }
