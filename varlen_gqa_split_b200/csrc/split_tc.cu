@@ -115,6 +115,32 @@ struct UnitDesc {
     long long pad;
 };
 
+// packed fp32 pairs (one instruction for two lanes' worth of FMA / add)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long ra, rb, rc, rd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    unsigned long long ra, rb, rd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // bounded mbarrier wait that also gives up when another role raised the stop flag
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *stop, const Params &p,
                                          unsigned long long factor = 1) {
@@ -703,18 +729,22 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                     whole_rows = __all_sync(0xffffffffu, (lo_c == 0 && width == kBN) || (width == 0 && !stale));
                     if (whole_rows) {
 #pragma unroll
-                        for (int cc = 0; cc < kBN; ++cc)
-                            mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(sv[cc >> 5][cc & 31]));
+                        for (int cc = 0; cc < kBN; cc += 2)
+                            mx4[(cc >> 1) & 3] = fmax3(mx4[(cc >> 1) & 3], __uint_as_float(sv[cc >> 5][cc & 31]),
+                                                       __uint_as_float(sv[cc >> 5][(cc + 1) & 31]));
                         if (width == 0) mx4[0] = mx4[1] = mx4[2] = mx4[3] = -INFINITY;
                         dead = width == 0;
                     } else {
                         // masked by selection, no branch per key
 #pragma unroll
-                        for (int cc = 0; cc < kBN; ++cc) {
-                            const bool keep = (unsigned)(cc - lo_c) < (unsigned)width;
-                            const uint32_t x = keep ? sv[cc >> 5][cc & 31] : 0xff800000u;   // -inf
-                            sv[cc >> 5][cc & 31] = x;
-                            mx4[cc & 3] = fmaxf(mx4[cc & 3], __uint_as_float(x));
+                        for (int cc = 0; cc < kBN; cc += 2) {
+                            const bool k0 = (unsigned)(cc - lo_c) < (unsigned)width;
+                            const bool k1 = (unsigned)(cc + 1 - lo_c) < (unsigned)width;
+                            const uint32_t x0 = k0 ? sv[cc >> 5][cc & 31] : 0xff800000u;   // -inf
+                            const uint32_t x1 = k1 ? sv[cc >> 5][(cc + 1) & 31] : 0xff800000u;
+                            sv[cc >> 5][cc & 31] = x0;
+                            sv[cc >> 5][(cc + 1) & 31] = x1;
+                            mx4[(cc >> 1) & 3] = fmax3(mx4[(cc >> 1) & 3], __uint_as_float(x0), __uint_as_float(x1));
                         }
                     }
                     mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * cs;
@@ -754,15 +784,18 @@ __global__ void __launch_bounds__(kThreads, 1) split_tc_kernel(const __grid_cons
                     const float nref = dead ? -INFINITY : (m_used == -INFINITY ? 0.f : -m_used);
                     const float csr = dead ? 0.f : cs;
                     uint32_t pk[kBN / 2];
-                    float l4[4] = {0.f, 0.f, 0.f, 0.f};
+                    float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    const float2 cs2 = make_float2(csr, csr), nr2 = make_float2(nref, nref);
 #pragma unroll
                     for (int i = 0; i < kBN / 2; ++i) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sv[i >> 4][(2 * i) & 31]), csr, nref));
-                        const float p1 = ex2(fmaf(__uint_as_float(sv[i >> 4][(2 * i + 1) & 31]), csr, nref));
-                        l4[i & 3] += p0 + p1;
-                        pk[i] = pack_bf16x2(p0, p1);
+                        const float2 x = ffma2(make_float2(__uint_as_float(sv[i >> 4][(2 * i) & 31]),
+                                                           __uint_as_float(sv[i >> 4][(2 * i + 1) & 31])),
+                                               cs2, nr2);
+                        const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+                        l2[i & 1] = fadd2(l2[i & 1], pp);
+                        pk[i] = pack_bf16x2(pp.x, pp.y);
                     }
-                    l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                    l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
                     if (!waited) {
                         if (!(ok = wwait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
                         tc::fence_after_sync();
