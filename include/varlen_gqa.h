@@ -133,7 +133,11 @@ typedef struct {
                               B_max); tensor-core (ctas, 1, 1)                    */
     int ctas;              /* tensor-core path: persistent blocks (0 on SIMT)    */
     int deterministic;     /* 1 if results are bitwise repeatable for this plan  */
-    int combine;           /* ATTN_COMBINE_KERNEL or ATTN_COMBINE_FUSED          */
+    int combine;           /* ATTN_COMBINE_KERNEL or ATTN_COMBINE_FUSED; 0 when
+                              no unit is ever split (one split per unit on the
+                              CUDA-core path; on the warp-MMA path, plans of
+                              units of <= 128 keys that fit one wave take one
+                              block per unit and write every row directly) */
     int combine_blocks;    /* combine-kernel blocks (0 unless a combine kernel runs) */
     int smem_bytes;        /* dynamic shared memory of the split kernel          */
     int num_sms;           /* SM count of the plan's device                      */

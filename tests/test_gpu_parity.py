@@ -295,6 +295,27 @@ def _packed_cases(B, values):
     return lq, lk
 
 
+@pytest.mark.parametrize("G,D", [(4, 64), (8, 128), (16, 128)])
+def test_direct_one_block_per_unit(G, D):
+    """Units of at most two tiles that fit one wave: the warp-MMA plan gives
+    block c unit c whole and launches no merge.  Every length edge of such a
+    plan (Lq 0, 1 and 2 with Lk 0, 1, 63, 64, 65, 127, 128, Lq > Lk, and
+    zero-length sequences padding B_max) against the oracle, with NaN
+    sentinels in the rows past cu_q."""
+    lq = [1, 1, 0, 2, 1, 2, 1, 1, 2, 0, 1, 0, 0]
+    lk = [0, 1, 5, 1, 63, 64, 65, 127, 128, 0, 128, 0, 0]
+    max_q = 2 if G <= 8 else 1
+    lq = [min(x, max_q) for x in lq]
+    sh = W.Shape("direct", B=len(lq), Hq=2 * G, Hkv=2, D=D, max_q=max_q, s_max=128)
+    batch = W.make_batch(sh, lq, lk, seed=53, gen_device="cuda")
+    plan = plan_for(sh)
+    assert plan.info["variant"] == MMA and plan.info["combine"] == 0 and plan.info["ctas"] == 2 * len(lq)
+    ref_o, ref_l = oracle_full(batch)
+    for _ in range(2):                                   # and a second call on the same plan
+        out, lse = run_gpu(plan, batch, extra_q_rows=3)
+        compare_full(out, lse, ref_o, ref_l, covered_rows(batch))
+
+
 @pytest.mark.parametrize("variant", [SIMT, MMA, TC])
 def test_exhaustive_small_lengths_placement(variant):
     """Every (Lq, Lk) combination with lengths in [0, 4] for 3 sequences (the
@@ -380,6 +401,9 @@ def test_plan_choices_follow_the_split_rule():
     assert pf.info["combine_blocks"] == 0
     tiny = plan_for(W.SHAPES["tiny"])                 # units of <= 2 tiles: one block each, none cut
     assert tiny.info["variant"] == MMA and tiny.info["ctas"] == 2
+    assert tiny.info["combine"] == 0 and tiny.info["combine_blocks"] == 0      # written directly, no merge
+    small = plan_for(W.Shape("small", B=300, Hq=8, Hkv=1, D=128, max_q=1, s_max=128))
+    assert small.info["combine"] == vg.ATTN_COMBINE_KERNEL                    # 300 units > one wave: shares
 
 
 # ------------------------------------------------------------ errors

@@ -36,6 +36,7 @@ struct attn_plan_s {
     int merge_bytes;           // tensor-core path: shared bytes of the merge area
     int qtile;                 // tensor-core path: query tokens per row tile
     int max_rt;                // tensor-core path: row tiles per sequence at most
+    int direct;                // warp-MMA path: one block per unit, no merge
     float *o_part;
     float2 *ml_part;
     unsigned long long wait_ns; // limit of one bounded wait in the kernels
@@ -236,6 +237,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     int qtile = max_q, max_rt = 1;
     size_t n_ticket = 0, n_part = 0, part_rows = 0;
     int merge_bytes = 0;
+    bool plan_direct = false;
     if (variant == ATTN_VARIANT_MMA || variant == ATTN_VARIANT_TC) {
         // persistent: about one block per SM, each with a deep load ring; the
         // split points follow the balanced per-block shares (nsplit and chunk
@@ -254,8 +256,14 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         // units of at most two tiles (s_max <= 128 keys): cutting one saves a
         // block at most one tile but adds a merge, so each unit gets its own
         // block (measured on the tiny workload: 14.3 against 16.4 us isolated)
-        if (!(o && o->ctas) && tiles_max <= 2)
-            ctas = std::min<long long>(ctas, std::max(1LL, (long long)B_max * Hkv * max_rt));
+        const long long units = (long long)B_max * Hkv * max_rt;
+        if (!(o && o->ctas) && tiles_max <= 2) ctas = std::min<long long>(ctas, std::max(1LL, units));
+        // ... and on the warp-MMA path, when those units fit one wave, block c
+        // simply takes unit c: no unit is ever cut, so no merge is launched
+        // and no schedule is computed speculatively (the direct write of the
+        // split-KV method, for the smallest calls)
+        const bool direct = !tcv && !(o && o->ctas) && tiles_max <= 2 && units <= sms;
+        if (direct) ctas = units;
         ctas = std::min<long long>(ctas, 65535);
         d.ctas = (int)ctas;
         auto smem_of = [&](int st) { return tcv ? tc_smem_need(D, st) : mma_smem_bytes(D, NT, st, d.ctas); };
@@ -291,9 +299,10 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
         const int want = o && o->combine ? o->combine
                                          : (tcv && d.deterministic && max_rt > 1 ? ATTN_COMBINE_FUSED
                                                                                   : ATTN_COMBINE_KERNEL);
-        d.combine = tcv ? want : ATTN_COMBINE_KERNEL;
+        d.combine = tcv ? want : (direct ? 0 : ATTN_COMBINE_KERNEL);
         if (d.combine == ATTN_COMBINE_FUSED && !d.deterministic) return ATTN_E_UNSUPPORTED;
         d.combine_blocks = d.combine == ATTN_COMBINE_KERNEL ? 2 * d.ctas * combine_slots_split((Hq / Hkv) * qtile, D) : 0;
+        plan_direct = direct;
         // per unit: tile claims (64-bit), parts written
         n_ticket = 3 * (size_t)B_max * Hkv * max_rt;
         n_part = 2 * (size_t)d.ctas;       // two partial slots per block
@@ -360,6 +369,7 @@ ATTN_EXPORT int attn_plan_ex(attn_plan_t *out, int B_max, int s_max, int Hq, int
     p->merge_bytes = merge_bytes;
     p->qtile = qtile;
     p->max_rt = max_rt;
+    p->direct = plan_direct ? 1 : 0;
     p->scale_log2 = (float)((1.0 / std::sqrt((double)D)) * 1.4426950408889634);
     p->wait_ns = o && o->wait_limit_us > 0 ? (unsigned long long)o->wait_limit_us * 1000ull : kDefaultWaitNs;
     if (cudaMalloc(&p->scratch, total) != cudaSuccess) {
@@ -503,6 +513,7 @@ int run_impl(attn_plan_t plan, const void *q, const void *k, const void *v, cons
     p.unit_cost = d.variant == ATTN_VARIANT_TC ? tc_unit_cost() : 0;
     p.qtile = plan->qtile;
     p.max_rt = plan->max_rt;
+    p.direct = plan->direct;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(d.grid_x, d.grid_y, d.grid_z);

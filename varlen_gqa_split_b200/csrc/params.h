@@ -36,6 +36,7 @@ struct Params {
                                // holding a cut unit's last part does
     int merge_bytes;           // tensor-core path: shared bytes of the merge area
     int ctas_max;              // tensor-core path: blocks of the launch (merge table size)
+    int direct;                // warp-MMA path: block c takes unit c whole (no cut units, no merge)
     int dynamic;               // tensor-core path: blocks sharing a cut unit claim its tiles
     int head_first;            // tensor-core path: schedule order for the fused merge (OrderedWalker)
     int done_per_part;         // tensor-core path: releases on `done` per written part

@@ -399,6 +399,60 @@ __device__ __forceinline__ bool block_share(const Params &p, int c, int C, int t
     return sh.b_first >= 0;                                 // always when lo < T
 }
 
+// Direct mode (plans whose units are at most two tiles and at most one per
+// SM): block c takes unit c = (b, hk) whole -- sequence b = c / Hkv, one row
+// tile -- so no unit is ever cut, every result is written by the split
+// kernel and no merge runs.  Same scan as block_share (each thread weighs a
+// run of sequences); the thread whose run holds b finds the unit's first
+// position.  Returns false for a block without a unit (b past B_max, or a
+// sequence without query tokens).
+__device__ __forceinline__ bool unit_share(const Params &p, int c, int tid, int nthreads, bool report,
+                                           long long *scan, long long *first, Share &sh) {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int per = (p.B_max + nthreads - 1) / nthreads;
+    const int b_lo = min(p.B_max, tid * per), b_hi = min(p.B_max, b_lo + per);
+    const int bc = c / p.Hkv, hk = c - bc * p.Hkv;
+    long long my = 0, w_c = 0, before_c = 0;                // run weight; unit c's weight; run weight before b_c
+    for (int b = b_lo; b < b_hi; ++b) {
+        const long long w = (long long)p.Hkv * seq_len(p, b, report).tpu;
+        if (b < bc) before_c += w;
+        if (b == bc) w_c = w / p.Hkv;
+        my += w;
+    }
+    long long incl = my;                                    // warp-inclusive scan
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) scan[warp] = incl;
+    if (tid == 0) first[0] = -1;
+    __syncthreads();
+    if (tid == 0) {
+        long long run = 0;
+        for (int w = 0; w < nthreads / 32; ++w) {
+            const long long x = scan[w];
+            scan[w] = run;
+            run += x;
+        }
+        first[2] = run;
+    }
+    __syncthreads();
+    sh.T = first[2];
+    if (bc >= b_lo && bc < b_hi && w_c > 0) {
+        first[0] = bc;
+        first[1] = incl - my + scan[warp] + before_c;       // tiles before sequence b_c
+        scan[0] = w_c;                                      // (every thread has read its scan entry)
+    }
+    __syncthreads();
+    sh.Ce = (int)gridDim.x;
+    sh.b_first = (int)first[0];
+    sh.pb_first = first[1];
+    sh.lo = sh.pb_first + hk * scan[0];
+    sh.hi = sh.lo + scan[0];
+    return bc < p.B_max && sh.b_first >= 0;
+}
+
 // The block's tiles in the order its producer loads them.  For every segment
 // of the block (OrderedWalker order) begin(seg, role) runs once, then
 // tile(seg, t, last) for each tile t of the unit the block takes -- `last`

@@ -58,9 +58,10 @@ struct MmaLayout {
     static constexpr int kStageBytes = 2 * kTileBytes;      // K + V
 };
 
-// PAGED: K and V come from a paged cache (block table); a separate
-// instantiation keeps the packed kernel free of that code
-template <int D, int NT, bool PAGED>
+// PAGED: K and V come from a paged cache (block table); DIRECT: block c takes
+// unit c whole (plans whose units all fit one wave of blocks, no merge).
+// Separate instantiations keep each kernel free of the code it does not run.
+template <int D, int NT, bool PAGED, bool DIRECT>
 __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                 const __grid_constant__ CUtensorMap tm_v,
                                                                 const Params p, const int stages) {
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
     // are hints: the L2 is coherent, so a prefetched line never hides a later
     // write, and the tensor map bounds every prefetch whatever the lengths
     // read.
-    if constexpr (!PAGED) {
+    if constexpr (!PAGED && !DIRECT) {         // (direct mode: every share is a whole unit, nothing to prefetch)
         Share sp;
         if (block_share(p, c, gridDim.x, tid, kThreads, false, scan, first, sp, true) && warp == kConsumerWarps)
             first_tiles(p, c, sp, kPrefetchBytes / L::kStageBytes, true, [&](const Segment &sg, int t) {
@@ -128,7 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
 
     // ------------------------------------------------------------ schedule
     Share sh;
-    if (!block_share(p, c, gridDim.x, tid, kThreads, c == 0, scan, first, sh)) return;
+    if (!(DIRECT ? unit_share(p, c, tid, kThreads, c == 0, scan, first, sh)
+                 : block_share(p, c, gridDim.x, tid, kThreads, c == 0, scan, first, sh)))
+        return;
     const long long lo = sh.lo, hi = sh.hi;
     const int b_first = sh.b_first;
     const long long pb_first = sh.pb_first;
@@ -506,14 +509,17 @@ __global__ void __launch_bounds__(kThreads, 1) split_mma_kernel(const __grid_con
 }
 
 template <int D, int NT>
-void *mma_kernel_ptr(bool paged) {
-    return paged ? reinterpret_cast<void *>(split_mma_kernel<D, NT, true>)
-                 : reinterpret_cast<void *>(split_mma_kernel<D, NT, false>);
+void *mma_kernel_ptr(bool paged, bool direct) {
+    if (direct)
+        return paged ? reinterpret_cast<void *>(split_mma_kernel<D, NT, true, true>)
+                     : reinterpret_cast<void *>(split_mma_kernel<D, NT, false, true>);
+    return paged ? reinterpret_cast<void *>(split_mma_kernel<D, NT, true, false>)
+                 : reinterpret_cast<void *>(split_mma_kernel<D, NT, false, false>);
 }
 
-void *pick(int D, int NT, bool paged) {
-    if (D == 64) return NT == 1 ? mma_kernel_ptr<64, 1>(paged) : mma_kernel_ptr<64, 2>(paged);
-    return NT == 1 ? mma_kernel_ptr<128, 1>(paged) : mma_kernel_ptr<128, 2>(paged);
+void *pick(int D, int NT, bool paged, bool direct) {
+    if (D == 64) return NT == 1 ? mma_kernel_ptr<64, 1>(paged, direct) : mma_kernel_ptr<64, 2>(paged, direct);
+    return NT == 1 ? mma_kernel_ptr<128, 1>(paged, direct) : mma_kernel_ptr<128, 2>(paged, direct);
 }
 
 }  // namespace
@@ -539,13 +545,13 @@ int mma_block_n() { return kBN; }
 int mma_threads() { return kThreads; }
 
 cudaError_t mma_prepare(int D, int NT, int stages, int ctas) {
-    for (bool paged : {false, true}) {
-        const cudaError_t e = cudaFuncSetAttribute(pick(D, NT, paged), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)mma_smem_bytes(D, NT, stages, ctas));
-        if (e != cudaSuccess) return e;
-    }
-    cudaError_t e = cudaSuccess;
-    if (e != cudaSuccess) return e;
+    for (bool paged : {false, true})
+        for (bool direct : {false, true}) {
+            const cudaError_t e =
+                cudaFuncSetAttribute(pick(D, NT, paged, direct), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)mma_smem_bytes(D, NT, stages, ctas));
+            if (e != cudaSuccess) return e;
+        }
     return combine_slots_prepare(D, ctas);
 }
 
@@ -569,8 +575,8 @@ cudaError_t launch_split_mma(const Params &p, const CUtensorMap &tm_k, const CUt
     int st = stages;
     void *split_args[] = {const_cast<CUtensorMap *>(&tm_k), const_cast<CUtensorMap *>(&tm_v),
                           const_cast<Params *>(&p), &st};
-    cudaError_t e = cudaLaunchKernelExC(&cfg, pick(p.D, NT, p.block_table != nullptr), split_args);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaLaunchKernelExC(&cfg, pick(p.D, NT, p.block_table != nullptr, p.direct != 0), split_args);
+    if (e != cudaSuccess || p.direct) return e;            // direct mode: no unit is cut, nothing to merge
     return launch_combine_slots(p, ctas, stream);
 }
 
