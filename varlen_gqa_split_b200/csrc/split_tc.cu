@@ -4,8 +4,9 @@
 // longer queries as several row tiles of the sequence, each its own unit.
 //
 // Same schedule as the warp-MMA kernel (schedule.cuh: equal shares of the
-// flattened 64-key tiles, cut units merged by the slot combine kernel; by
-// default the shares stay static on this path, without run-time claims), but
+// flattened 64-key tiles; by default the shares stay static on this path,
+// without run-time claims; cut units are merged by the slot combine kernel,
+// or, instantiated with FUSED, by the block holding each one's last part), but
 // the G query heads times the q_len query tokens of a unit form the M = 128
 // side of real tensor-core tiles (kernbench2 docs/adr-proposed commit log,
 // GQA entry: G folded into the matmul M dimension; every K/V byte is read
