@@ -54,7 +54,7 @@ def _run_paged(plan, batch, pc):
 
 
 @pytest.mark.parametrize("page_size", [8, 16, 64, 256])
-@pytest.mark.parametrize("variant,Hq,max_q", [(MMA, 16, 1), (MMA, 16, 4), (TC, 32, 8), (SIMT, 16, 2)])
+@pytest.mark.parametrize("variant,Hq,max_q", [(MMA, 16, 1), (MMA, 16, 4), (TC, 32, 8), (TC, 32, 40), (SIMT, 16, 2)])
 def test_paged_parity(variant, Hq, max_q, page_size):
     sh, batch = _edge_batch(Hq, max_q)
     pc = W.paginate(batch.k, batch.v, batch.cu_k, sh.B, page_size, sh.s_max, seed=page_size, extra_cols=2)
@@ -83,13 +83,18 @@ def test_paged_fused_cache_layout(variant):
 @pytest.mark.parametrize("variant", [MMA, TC])
 def test_paged_split_units_and_block_counts(variant):
     """Few blocks over long sequences: units cut across blocks, run-time
-    claims and the slot combine, all through the page table."""
+    claims, the slot combine and (tcgen05) the fused merge, all through the
+    page table."""
     Hq, max_q = (16, 1) if variant == MMA else (32, 8)
     sh = W.Shape("paged_long", B=3, Hq=Hq, Hkv=4, D=128, max_q=max_q, s_max=9000)
     batch = W.make_batch(sh, [1, max_q, min(2, max_q)], [9000, 4097, 3001], seed=41, gen_device="cuda")
     pc = W.paginate(batch.k, batch.v, batch.cu_k, sh.B, 16, sh.s_max, seed=5)
     ref_o, ref_l = oracle_full(batch)
-    for kw in ({"ctas": 7}, {"ctas": 7, "deterministic": 1}, {"ctas": 7, "deterministic": -1}, {}):
+    kws = [{"ctas": 7}, {"ctas": 7, "deterministic": 1}, {"ctas": 7, "deterministic": -1}, {}]
+    if variant == TC:
+        # the fused merge (the block holding each cut unit's last part merges it) on pages
+        kws.append({"ctas": 7, "combine": vg.ATTN_COMBINE_FUSED})
+    for kw in kws:
         plan = plan_for(sh, variant=variant, **kw)
         out, lse = _run_paged(plan, batch, pc)
         assert plan.check_error() == 0
