@@ -171,12 +171,12 @@ struct SegWalker {
 // balancing can even out the blocks' finishing times without delaying any
 // block's own units.  `head_first` (static shares with the fused merge, in
 // which the block holding a cut unit's last part merges it) orders them so
-// that the merge never waits: the unit cut at the share's end first (a head
+// that a merge seldom waits: the unit cut at the share's end first (a head
 // or middle part, which some later block merges), then the block's own
 // units, then the unit cut at its start (whose last part this block may
 // hold, the other parts having been streamed first by their blocks).
-// HF: head-first order compiled in (the tensor-core kernel); the kernels that
-// never use it keep the plain walker.
+// HF: head-first order compiled in (the tcgen05 kernel with the fused
+// merge); the kernels that never use it keep the plain walker.
 template <bool HF = false>
 struct OrderedWalker {
     SegWalker wk;
