@@ -178,7 +178,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
 
 // ------------------------------------------------------------ TMA
 
-// 3-D tiled bulk tensor load (no multicast) into shared memory, completing
+// 3-D tiled bulk tensor load into shared memory, completing
 // `bar`'s transaction count.  coords: {c0 innermost, c1, c2}.
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
                                             int c0, int c1, int c2, uint64_t policy) {
@@ -225,7 +225,7 @@ __device__ __forceinline__ void tma_load_5d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
-// 1-D bulk copy global -> shared (no multicast), completing `bar`'s
+// 1-D bulk copy global -> shared, completing `bar`'s
 // transaction count.  dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(

@@ -11,7 +11,7 @@
 // Producer: the whole warp walks the block's units in step (lane 0 takes the
 // claims and keeps the stage bookkeeping, each lane issues one box) and
 // streams their K and V tiles (64 keys x D, one box per tensor covering every
-// D-half) with cp.async.bulk.tensor (no multicast) into a ring of
+// D-half) with cp.async.bulk.tensor (this CTA only) into a ring of
 // shared-memory stages in the 128-byte swizzled layout, one mbarrier per
 // stage, L2 evict-first.  The ring runs across unit boundaries, so the next
 // unit's loads are in flight while the current unit finishes.  A tile whose
